@@ -1,0 +1,24 @@
+"""Shared pytest configuration: the ``gpu`` marker and the repo root on sys.path.
+
+Tests marked ``gpu`` need a CUDA device and the built CUDA library; everything else runs on
+CPU (``pytest -m "not gpu"``)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a) and the built library")
+    config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+@pytest.fixture(scope="session")
+def oracle_mod():
+    import oracle
+    oracle.lib()
+    return oracle

@@ -1,0 +1,277 @@
+"""Pins for the oracle's optimizer step (CPU only).
+
+The abstract of "8-bit Optimizers via Block-wise Quantization" (quoted on the blog.csdn.net
+bitsandbytes guide, section 2) names the stateful optimizers -- SGD with momentum (smoothed
+sum) and Adam (smoothed and squared sums) -- and says the 8-bit optimizers are a drop-in
+replacement that keeps 32-bit performance.  The page "bitsandbytes深度解析", section
+"优化器模块深度分析", lists AdamW8bit, Adam8bit, SGD8bit and Lion8bit.  So with quantization
+out of the way (32-bit state) the oracle's step must agree with torch.optim's AdamW, Adam and
+SGD, which these tests run in float64 as an independent reference; Lion is pinned by its
+closed-form special cases.  The 8-bit path is pinned as "dequantize -> the same update ->
+nearest-code requantize" against torch and an exact brute-force nearest code.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+HP = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+
+
+def _f(x):
+    """binary32 value of a hyper-parameter, as the oracle sees it."""
+    return float(np.float32(x))
+
+
+def _close(got, want, scale, rtol=2e-6, ulps=4):
+    """|got - want| <= rtol*|want| + ulps * ulp32(scale): fp32 rounding against an fp64 reference,
+    with an absolute floor set by the size of the operands (cancellation leaves small results)."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    tol = rtol * np.abs(want) + ulps * np.spacing(np.abs(np.asarray(scale, np.float32))).astype(np.float64)
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), (np.nonzero(bad)[0][:5], got[bad][:5], want[bad][:5])
+
+
+def _grads(n, steps, seed, tiny_fraction=0.05):
+    rng = np.random.default_rng(seed)
+    gs = []
+    for _ in range(steps):
+        g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+        tiny = rng.random(n) < tiny_fraction  # gradients where eps matters
+        g[tiny] *= 1e-5
+        gs.append(g)
+    return gs
+
+
+def _torch_run(opt_cls, p0, grads, **kw):
+    p = torch.nn.Parameter(torch.from_numpy(p0.astype(np.float64)))
+    opt = opt_cls([p], **kw)
+    for g in grads:
+        p.grad = torch.from_numpy(g.astype(np.float64))
+        opt.step()
+    return p.detach().numpy(), opt.state[p]
+
+
+@pytest.mark.parametrize("wd", [0.0, 0.01])
+def test_adamw_32bit_matches_torch(oracle_mod, wd):
+    n, steps = 5000, 10
+    p0 = (np.random.default_rng(0).standard_normal(n) * 0.02).astype(np.float32)
+    grads = _grads(n, steps, 1)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    hp = dict(HP, weight_decay=wd)
+    for t, g in enumerate(grads, 1):
+        oracle_mod.step_tensor("adamw", p, g, m, v, None, None, None, None, 2048, step=t, **hp)
+    pt, st = _torch_run(torch.optim.AdamW, p0, grads, lr=_f(hp["lr"]), betas=(_f(0.9), _f(0.999)),
+                        eps=_f(1e-8), weight_decay=_f(wd), foreach=False)
+    _close(p, pt, np.abs(p0) + hp["lr"] * steps)  # operand scale: p0 and the summed updates
+    _close(m, st["exp_avg"].numpy(), np.max(np.abs(m)), rtol=2e-5)
+    _close(v, st["exp_avg_sq"].numpy(), np.max(v), rtol=2e-5)
+
+
+def test_adamw_first_step_closed_form(oracle_mod):
+    """P5: from zero state, step 1 moves p by lr * g / (|g| + eps) after the decoupled decay."""
+    n = 4096
+    rng = np.random.default_rng(5)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    oracle_mod.step_tensor("adamw", p, g, m, v, None, None, None, None, 2048, step=1, **HP)
+    lr, wd, eps = _f(HP["lr"]), _f(HP["weight_decay"]), _f(HP["eps"])
+    g64 = g.astype(np.float64)
+    want = p0 * (1 - lr * wd) - lr * g64 / (np.abs(g64) + eps)
+    _close(p, want, np.abs(p0) + lr, rtol=0)
+
+
+def test_adam_l2_matches_torch(oracle_mod):
+    n, steps = 3000, 6
+    p0 = (np.random.default_rng(2).standard_normal(n) * 0.02).astype(np.float32)
+    grads = _grads(n, steps, 3)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    hp = dict(HP, weight_decay=0.1)
+    for t, g in enumerate(grads, 1):
+        oracle_mod.step_tensor("adam", p, g, m, v, None, None, None, None, 256, step=t, **hp)
+    pt, _ = _torch_run(torch.optim.Adam, p0, grads, lr=_f(1e-3), betas=(_f(0.9), _f(0.999)), eps=_f(1e-8),
+                       weight_decay=_f(0.1), foreach=False)
+    _close(p, pt, np.abs(p0) + 1e-3 * steps)
+
+
+@pytest.mark.parametrize("wd", [0.0, 1e-2])
+def test_momentum_matches_torch_sgd(oracle_mod, wd):
+    n, steps = 3000, 8
+    p0 = (np.random.default_rng(4).standard_normal(n) * 0.02).astype(np.float32)
+    grads = _grads(n, steps, 5)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    for t, g in enumerate(grads, 1):
+        oracle_mod.step_tensor("momentum", p, g, m, None, None, None, None, None, 2048, step=t,
+                               lr=1e-2, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=wd)
+    pt, st = _torch_run(torch.optim.SGD, p0, grads, lr=_f(1e-2), momentum=_f(0.9), weight_decay=_f(wd),
+                        foreach=False)
+    _close(p, pt, np.abs(p0) + 1e-2 * np.abs(st["momentum_buffer"].numpy()).max() * steps, rtol=1e-6)
+    _close(m, st["momentum_buffer"].numpy(), np.max(np.abs(m)), rtol=1e-5)
+
+
+def test_momentum_first_step(oracle_mod):
+    """P6: from zero state, momentum SGD's first step is p - lr * g, to one rounding."""
+    n = 1000
+    p0 = np.linspace(-1, 1, n).astype(np.float32)
+    g = np.linspace(2, -3, n).astype(np.float32)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    oracle_mod.step_tensor("momentum", p, g, m, None, None, None, None, None, 256, step=1,
+                           lr=0.5, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=0.0)
+    np.testing.assert_array_equal(m, g)
+    np.testing.assert_array_equal(p, (p0 - np.float32(0.5) * g).astype(np.float32))
+
+
+def test_lion_sign_update(oracle_mod):
+    """P6: Lion moves each parameter by exactly -lr*sign(b1*m + (1-b1)*g) after the decay, and
+    the state becomes the b2-smoothed gradient."""
+    n, lr, wd = 4000, 1e-4, 0.1
+    rng = np.random.default_rng(6)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    m0 = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    g[:10] = 0.0
+    m0[:10] = 0.0  # c == 0 -> no move
+    p, m = p0.copy(), m0.copy()
+    oracle_mod.step_tensor("lion", p, g, m, None, None, None, None, None, 2048, step=3,
+                           lr=lr, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=wd)
+    decayed = (p0 * np.float32(1 - _f(lr) * _f(wd))).astype(np.float32)
+    step = (decayed.astype(np.float64) - p) / _f(lr)
+    c64 = _f(0.9) * m0.astype(np.float64) + (1 - _f(0.9)) * g
+    clear = np.abs(c64) > 1e-9
+    np.testing.assert_allclose(step[clear], np.sign(c64[clear]), atol=1e-3)
+    assert np.all(p[:10] == decayed[:10])
+    m64 = _f(0.99) * m0.astype(np.float64) + (1 - _f(0.99)) * g
+    np.testing.assert_allclose(m, m64, rtol=1e-6, atol=1e-12)
+
+
+# ----------------------------------------------------------------------- 8-bit state path
+def _dequant(code, q, absmax, n, B):
+    return code[q].astype(np.float64) * np.repeat(absmax.astype(np.float64), B)[:n]
+
+
+def _nearest_exact(code, xn):
+    c64 = code.astype(np.float64)
+    hi = np.clip(np.searchsorted(c64, xn, side="left"), 1, len(code) - 1)
+    lo = hi - 1
+    return np.where(c64[hi] - xn < xn - c64[lo], hi, lo), np.minimum(c64[hi] - xn, xn - c64[lo])
+
+
+def test_8bit_first_step_equals_32bit(oracle_mod):
+    """From zero state the dequantized state is exactly zero, so the 8-bit and 32-bit paths give
+    bit-identical parameters at step 1; the stored 8-bit state is the nearest code of m/absmax."""
+    n, B = 65536 + 333, 2048
+    rng = np.random.default_rng(8)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    c1, c2 = oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    p8 = p0.copy()
+    q1 = np.full(n, 127, np.uint8)
+    q2 = np.zeros(n, np.uint8)
+    a1 = np.zeros(nb, np.float32)
+    a2 = np.zeros(nb, np.float32)
+    oracle_mod.step_tensor("adamw", p8, g, q1, q2, a1, a2, c1, c2, B, step=1, **HP)
+    p32 = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    oracle_mod.step_tensor("adamw", p32, g, m, v, None, None, None, None, B, step=1, **HP)
+    np.testing.assert_array_equal(p8, p32)
+    # requantized state: block absmax of the 32-bit state, then the nearest code
+    for a, q, s, code in ((a1, q1, m, c1), (a2, q2, v, c2)):
+        want_a = np.array([np.max(np.abs(s[i:i + B])) for i in range(0, n, B)], np.float32)
+        np.testing.assert_array_equal(a, want_a)
+        xn = (s / np.repeat(want_a, B)[:n]).astype(np.float32).astype(np.float64)
+        qq, _ = _nearest_exact(code, xn)
+        np.testing.assert_array_equal(q, qq)
+
+
+def test_8bit_step_from_quantized_state_matches_torch(oracle_mod):
+    """A step from a random 8-bit state equals torch's AdamW run from the dequantized state; the
+    new state is the nearest code of the new moments (checked away from decision boundaries)."""
+    n, B, t = 8192 + 77, 2048, 7
+    rng = np.random.default_rng(9)
+    c1, c2 = oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    q1 = rng.integers(0, 256, n).astype(np.uint8)
+    q2 = rng.integers(0, 256, n).astype(np.uint8)
+    a1 = rng.uniform(1e-4, 1e-3, nb).astype(np.float32)
+    a2 = rng.uniform(1e-8, 1e-6, nb).astype(np.float32)
+    m0 = _dequant(c1, q1, a1, n, B)
+    v0 = _dequant(c2, q2, a2, n, B)
+    p = p0.copy()
+    oracle_mod.step_tensor("adamw", p, g, q1, q2, a1, a2, c1, c2, B, step=t, **HP)
+
+    tp = torch.nn.Parameter(torch.from_numpy(p0.astype(np.float64)))
+    opt = torch.optim.AdamW([tp], lr=_f(1e-3), betas=(_f(0.9), _f(0.999)), eps=_f(1e-8),
+                            weight_decay=_f(0.01), foreach=False)
+    opt.state[tp] = {"step": torch.tensor(float(t - 1)), "exp_avg": torch.from_numpy(m0.copy()),
+                     "exp_avg_sq": torch.from_numpy(v0.copy())}
+    tp.grad = torch.from_numpy(g.astype(np.float64))
+    opt.step()
+    _close(p, tp.detach().numpy(), np.abs(p0) + 1e-3, rtol=1e-6)
+    m1 = opt.state[tp]["exp_avg"].numpy()
+    v1 = opt.state[tp]["exp_avg_sq"].numpy()
+    for a, q, s, code in ((a1, q1, m1, c1), (a2, q2, v1, c2)):
+        want_a = np.array([np.max(np.abs(s[i:i + B])) for i in range(0, n, B)])
+        np.testing.assert_allclose(a, want_a, rtol=1e-6)
+        xn = s / np.repeat(want_a, B)[:n]
+        qq, margin = _nearest_exact(code, xn)
+        far = margin > 1e-5 * np.maximum(np.abs(xn), 1e-7)  # not near a decision boundary
+        assert far.mean() > 0.99
+        np.testing.assert_array_equal(q[far], qq[far])
+
+
+def test_zero_gradient_zero_state_stays(oracle_mod):
+    """P6: zero gradient on zero 8-bit state keeps code(0) and absmax 0."""
+    n, B = 5000, 2048
+    c1, c2 = oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    p = np.ones(n, np.float32)
+    q1 = np.full(n, 127, np.uint8)
+    q2 = np.zeros(n, np.uint8)
+    a1 = np.zeros(nb, np.float32)
+    a2 = np.zeros(nb, np.float32)
+    oracle_mod.step_tensor("adamw", p, np.zeros(n, np.float32), q1, q2, a1, a2, c1, c2, B, step=1,
+                           lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0)
+    assert np.all(q1 == 127) and np.all(q2 == 0) and np.all(a1 == 0) and np.all(a2 == 0)
+    assert np.all(p == 1.0)
+
+
+def test_state_bytes_per_param():
+    """P8: 8-bit Adam keeps two one-byte codes per parameter (2 B/param of state, vs 8 B for two
+    fp32 moments: the 75% reduction of the bitsandbytes skill page, Workflow 3), plus one fp32
+    absmax per block per state."""
+    n, B = 7_000_000_000, 2048
+    state8 = 2 * n + 2 * 4 * ((n + B - 1) // B)
+    state32 = 8 * n
+    assert abs(state8 / n - 2.0) < 0.01
+    assert abs(1 - state8 / state32 - 0.75) < 0.002
+
+
+def test_bf16_gradients_are_widened_exactly(oracle_mod):
+    n = 3000
+    rng = np.random.default_rng(11)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    gt = torch.from_numpy((rng.standard_normal(n) * 1e-3).astype(np.float32)).to(torch.bfloat16)
+    bits = gt.view(torch.int16).numpy().view(np.uint16)
+    outs = []
+    for g in (bits, gt.float().numpy()):
+        p = p0.copy()
+        m = np.zeros(n, np.float32)
+        v = np.zeros(n, np.float32)
+        oracle_mod.step_tensor("adamw", p, g, m, v, None, None, None, None, 2048, step=1, **HP)
+        outs.append(p)
+    np.testing.assert_array_equal(outs[0], outs[1])
