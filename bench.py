@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the fused 8-bit optimizer step (one JSON line on rank 0).
+
+Default workload: 8-bit AdamW on the 7B Llama-shaped list (291 tensors, 6,738,415,616 fp32
+parameters, bf16 gradients ~N(0,1e-3), signed / unsigned dynamic codes for m / v, blocksize 2048,
+32-bit state for the token embedding; seed 4).  One step = one ``bnbq_step_8bit`` call = one
+kernel launch over the whole list.  Inputs live in HBM (about 96 GB of traffic per step, far
+above the 126 MB L2, so no L2 flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+``value``: parameters stepped per second over all ranks (each rank steps its own list: weak
+scaling, no collective on the data path).  ``e2e``: the same metric through the public API with
+the step's gradients copied from pinned host memory every step and the device flag word read
+back.  ``roofline``: algorithmic bytes of one launch / the launch's average CUDA-event duration,
+against the measured HBM copy bandwidth.  ``cpu_baseline``: the CPU oracle on a bounded sample.
+``--impl reference`` times that oracle alone (the slow reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "8-bit AdamW step params/s and achieved HBM GB/s (% of B200 HBM roofline), 1 GPU"
+WORKLOADS = {
+    # name: (shape, optimizer, seed, hyper-parameters, (outlier fraction, outlier scale))
+    "llama7b_adamw": ("llama7b", "adamw", 4, dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
+                      (0.0, 1.0)),
+    "gpt2_adamw": ("gpt2_1p5b", "adamw", 2, dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
+                   (0.0, 1.0)),
+    "llama7b_lion": ("llama7b", "lion", 3, dict(lr=1e-4, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=0.1),
+                     (1e-4, 100.0)),
+    "llama7b_momentum": ("llama7b", "momentum", 3, dict(lr=1e-2, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=0.0),
+                         (1e-4, 100.0)),
+    # one decoder layer (202M params, ~3 GB): the size used for ncu captures
+    "llama7b_layer_adamw": ("llama7b_layer", "adamw", 4,
+                            dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01), (0.0, 1.0)),
+}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "block_wise_bit_b200", "csrc", f) for f in
+                  ("bnbq_step.cu", "bnbq_device.cuh", "bnbq_internal.h")]
+
+
+def algorithmic_bytes(lay, optim: str, g_bytes: int = 2) -> int:
+    """Minimum HBM traffic of one step over the list: p read+write (8 B), g read, each state
+    read+write (1+1 B per 8-bit code, 4+4 B per fp32 moment), each 8-bit block scale read+write."""
+    two = optim in ("adamw", "adam")
+    ns = 2 if two else 1
+    total = 0
+    B = lay.blocksize
+    for s, bits in zip(lay.specs, lay.state_bits):
+        if bits == 8:
+            total += s.numel * (8 + g_bytes + 2 * ns) + ((s.numel + B - 1) // B) * 8 * ns
+        else:
+            total += s.numel * (8 + g_bytes + 8 * ns)
+    return total
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_per_launch(workload: str, n_params: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (scaled from the captured case by parameters processed); else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload.replace("_layer", "")) or d.get(workload)
+    if not e or e.get("kernel_src_sha") != kernel_source_sha():
+        return None
+    return int(round(e["dram_bytes_per_param"] * n_params))
+
+
+# ------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.uuid = device_uuid
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.split(",") for ln in self.file.read().strip().splitlines() if ln.count(",") >= 8]
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle leg
+def oracle_rate(shape: str, optim: str, hp: dict, elements8: int, threads: int, steps: int = 1):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload: ``elements8``
+    elements with 8-bit state plus the list's share of 32-bit-state elements, split over
+    ``threads`` threads (ctypes releases the GIL).  Returns (params/s, seconds, sample text)."""
+    import oracle
+    from block_wise_bit_b200 import workloads as W
+    B = 2048
+    lay = W.Layout.build(W.SHAPES[shape](), B)
+    two = optim in ("adamw", "adam")
+    frac32 = lay.n32 / max(1, lay.n_params)
+    n8 = (elements8 // B) * B
+    n32 = int(n8 * frac32 / max(1e-12, 1 - frac32)) // 4 * 4
+    rng = np.random.default_rng(0)
+
+    def arrays(n, bits):
+        p = (rng.standard_normal(n) * 0.02).astype(np.float32)
+        g = (rng.standard_normal(n) * 1e-3).astype(np.float32).view(np.uint32)
+        g = ((g + 0x7FFF + ((g >> 16) & 1)) >> 16).astype(np.uint16)  # bf16 bits (round to nearest even)
+        if bits == 8:
+            nb = (n + B - 1) // B
+            return dict(p=p, g=g, s1=rng.integers(0, 256, n).astype(np.uint8),
+                        s2=rng.integers(0, 256, n).astype(np.uint8) if two else None,
+                        a1=np.full(nb, 1e-3, np.float32), a2=np.full(nb, 1e-6, np.float32) if two else None)
+        return dict(p=p, g=g, s1=np.zeros(n, np.float32), s2=np.zeros(n, np.float32) if two else None,
+                    a1=None, a2=None)
+
+    work = [(arrays(n8, 8), n8)] + ([(arrays(n32, 32), n32)] if n32 else [])
+    c1, c2 = oracle.code_dynamic_signed(), oracle.code_dynamic_unsigned()
+    jobs = []
+    for arrs, n in work:
+        nb = (n + B - 1) // B
+        per = (nb + threads - 1) // threads
+        for t0 in range(0, nb, per):
+            jobs.append((arrs, (t0, min(nb, t0 + per))))
+
+    def run(job, t):
+        arrs, rng_ = job
+        oracle.step_tensor(optim, arrs["p"], arrs["g"], arrs["s1"], arrs["s2"], arrs["a1"], arrs["a2"], c1,
+                           c2 if two else None, B, step=t, block_range=rng_, **hp)
+
+    oracle.lib()
+    t0 = time.perf_counter()
+    for t in range(1, steps + 1):
+        ths = [threading.Thread(target=run, args=(j, t)) for j in jobs]
+        for th in ths:
+            th.start()
+        for th in ths:
+            th.join()
+    dt = time.perf_counter() - t0
+    sample = (f"{n8} 8-bit-state + {n32} 32-bit-state elements of the {shape} {optim} step "
+              f"(the list's 32-bit share), synthetic inputs, {steps} step(s), {threads} threads")
+    return (n8 + n32) * steps / dt, dt, sample
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# -------------------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama7b_adamw")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="8-bit elements in the CPU oracle sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS[args.workload]
+
+    from block_wise_bit_b200 import workloads as W
+    lay = W.Layout.build(W.SHAPES[shape](), 2048)
+    config = {"workload": f"{args.workload}8bit", "list": shape, "tensors": len(lay.specs),
+              "params": lay.n_params, "params_8bit_state": lay.n8, "params_32bit_state": lay.n32,
+              "blocksize": 2048, "grad_dtype": "bf16", "optimizer": optim, **hp,
+              "l2": "inputs far larger than the 126 MB L2 (no flush needed)"}
+    base = {"metric": METRIC, "unit": "params/s", "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded normal inputs, no weights)",
+            "config": config}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        threads = cpu_threads()
+        per_step = max(2048, args.cpu_sample // 4)
+        oracle_rate(shape, optim, hp, 2048 * threads, threads, 1)  # warm the library / pages
+        for _ in range(args.warmup):
+            oracle_rate(shape, optim, hp, per_step, threads, 1)
+        rates, secs = [], []
+        for _ in range(args.steps):
+            r, dt, sample = oracle_rate(shape, optim, hp, per_step, threads, 1)
+            rates.append(r)
+            secs.append(dt)
+        total = sum(secs)
+        value = float(statistics.median(rates))
+        out = dict(base, impl="reference", value=value, n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                   ms_per_step=1e3 * total / args.steps,
+                   cpu_baseline={"value": value, "unit": "params/s", "cores": threads, "kind": "oracle",
+                                 "sample": sample + " per step"},
+                   e2e={"value": value, "unit": "params/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+        print(json.dumps(out))
+        return
+
+    import torch
+    import torch.distributed as dist
+    import block_wise_bit_b200 as bq
+    from block_wise_bit_b200.optim import FlatStateList
+
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bq.lib()
+
+    fl = FlatStateList(lay, optim, dev, g_dtype=torch.bfloat16)
+    for i, spec in enumerate(lay.specs):
+        fl.entries[i].p.copy_(W.normal(spec.numel, 0.02, dev, shape, seed, rank, i, "p"))
+        W.grad_fill_(fl.entries[i].g, 1e-3, ofrac, oscale, shape, seed, rank, i, "g")
+    torch.cuda.synchronize()
+    bq.bnbq_device_flags(clear=True)
+
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        fl.step(t, **hp)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    stream = torch.cuda.current_stream(dev)
+    k_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for k in range(args.steps):
+        t += 1
+        k_start[k].record(stream)
+        fl.step(t, **hp)
+        k_end[k].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+
+    total_ms = ev0.elapsed_time(ev1)
+    launch_ms = [a.elapsed_time(b) for a, b in zip(k_start, k_end)]
+    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = lay.n_params * args.steps * world / (total_ms / 1e3)
+    flags = bq.bnbq_device_flags(clear=True)
+
+    alg = algorithmic_bytes(lay, optim, 2)
+    peak, peak_kind = measured_peaks()
+    achieved = alg / (avg_launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload, lay.n_params),
+                "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes_per_launch": alg,
+                "kernel": f"step_kernel<{optim}, 2048>", "avg_launch_ms": round(avg_launch_ms, 4),
+                "min_launch_ms": round(min(launch_ms), 4), "max_launch_ms": round(max(launch_ms), 4)}
+
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        g_host = torch.empty(fl.g.numel(), dtype=fl.g.dtype, pin_memory=True)
+        g_host.copy_(fl.g)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            t += 1
+            fl.g.copy_(g_host, non_blocking=True)
+            fl.step(t, **hp)
+            flags |= bq.bnbq_device_flags()  # device -> host read of the step's status word
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": lay.n_params * args.e2e_steps * world / (e_ms / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": g_host.numel() * g_host.element_size(), "d2h_bytes_per_step": 4,
+               "steps": args.e2e_steps}
+        del g_host
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = cpu_threads()
+        r, dt, sample = oracle_rate(shape, optim, hp, args.cpu_sample, threads, 1)
+        cpu = {"value": r, "unit": "params/s", "cores": threads, "kind": "oracle", "sample": sample,
+               "seconds": round(dt, 2)}
+
+    if rank == 0:
+        out = dict(base, value=value, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                   ms_per_step=round(ms_per_step, 4), roofline=roofline, cpu_baseline=cpu, e2e=e2e,
+                   gpu_launches=args.steps, clocks=clk, device_flags=flags,
+                   hbm_gbs_algorithmic=round(alg * args.steps / (total_ms / 1e3) / 1e9 * world, 1))
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

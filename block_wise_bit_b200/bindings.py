@@ -1,0 +1,237 @@
+"""ctypes binding of include/bnbq.h (libbnbq.so, built for sm_100a).
+
+Argument marshalling only: every step of quantization, dequantization and the optimizer step
+runs in the CUDA kernels of the library.  torch supplies device memory and the current stream.
+There is no fallback: if the library is missing or the tensors are not on a CUDA device, the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+from . import build as _build
+
+OK, EINVAL, EUNSUPPORTED, ECUDA = 0, 1, 2, 3
+F32, BF16 = 0, 1
+ADAMW, ADAM, LION, MOMENTUM = 0, 1, 2, 3
+OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM}
+CODE_DYNAMIC_SIGNED, CODE_DYNAMIC_UNSIGNED, CODE_NF4, CODE_LINEAR = 0, 1, 2, 3
+CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DYNAMIC_UNSIGNED,
+              "nf4": CODE_NF4, "linear": CODE_LINEAR}
+FLAG_BAD_CODE, FLAG_NONFINITE = 0x1, 0x2
+
+EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_codebook",
+            "bnbq_code_size", "bnbq_check_codebook", "bnbq_device_flags", "bnbq_last_error", "bnbq_release",
+            "bnbq_version"]
+
+
+class BnbqError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"bnbq status {status}: {msg}")
+        self.status = status
+
+
+class CTensor(ctypes.Structure):
+    """bnbq_tensor"""
+    _fields_ = [("p", ctypes.c_void_p), ("g", ctypes.c_void_p), ("state1", ctypes.c_void_p),
+                ("state2", ctypes.c_void_p), ("absmax1", ctypes.c_void_p), ("absmax2", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("g_dtype", ctypes.c_int32), ("state_bits", ctypes.c_int32)]
+
+
+class CHParams(ctypes.Structure):
+    """bnbq_hparams"""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libbnbq.so (building it with nvcc first if it is missing or stale and nvcc exists)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if build_if_missing:
+            try:
+                path = _build.build()
+            except RuntimeError:
+                if not os.path.exists(path):
+                    raise
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library {path} is not built (python -m block_wise_bit_b200.build)")
+        L = ctypes.CDLL(path)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.bnbq_quantize_blockwise.argtypes = [vp, i32, vp, i32, i64, i32, vp, vp, vp]
+        L.bnbq_dequantize_blockwise.argtypes = [vp, i32, vp, vp, i64, i32, vp, i32, vp]
+        L.bnbq_step_8bit.argtypes = [i32, ctypes.POINTER(CTensor), i32, ctypes.POINTER(CHParams), i32, vp, vp,
+                                     i32, vp]
+        for f in ("bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit",
+                  "bnbq_check_codebook", "bnbq_device_flags"):
+            getattr(L, f).restype = i32
+        L.bnbq_codebook.argtypes = [i32, vp]
+        L.bnbq_codebook.restype = i32
+        L.bnbq_code_size.argtypes = [i32]
+        L.bnbq_code_size.restype = i32
+        L.bnbq_check_codebook.argtypes = [vp, i32]
+        L.bnbq_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        L.bnbq_last_error.restype = ctypes.c_char_p
+        L.bnbq_last_error.argtypes = []
+        L.bnbq_release.restype = None
+        L.bnbq_release.argtypes = []
+        L.bnbq_version.restype = ctypes.c_char_p
+        L.bnbq_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != OK:
+        raise BnbqError(status, lib().bnbq_last_error().decode())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_id(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+# ------------------------------------------------------------------------------------ codebooks
+def bnbq_codebook(kind: str | int) -> torch.Tensor:
+    """Host-side construction of a codebook (CPU float32 tensor)."""
+    k = CODE_KINDS[kind] if isinstance(kind, str) else int(kind)
+    size = lib().bnbq_code_size(k)
+    if size < 0:
+        raise ValueError(f"unknown codebook kind {kind}")
+    out = torch.empty(size, dtype=torch.float32)
+    if lib().bnbq_codebook(k, ctypes.c_void_p(out.data_ptr())) != size:
+        raise ValueError(f"codebook {kind} failed")
+    return out
+
+
+def bnbq_check_codebook(code: torch.Tensor) -> None:
+    c = code.detach().to("cpu", torch.float32).contiguous()
+    _check(lib().bnbq_check_codebook(ctypes.c_void_p(c.data_ptr()), c.numel()))
+
+
+# --------------------------------------------------------------------------- quantize / dequant
+def bnbq_quantize_blockwise(code: torch.Tensor, A: torch.Tensor, blocksize: int = 2048,
+                            absmax: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                            stream=None):
+    """Return (absmax float32[ceil(n/B)], codes uint8[n] or packed uint8[ceil(n/2)] for 16 codes)."""
+    n = A.numel()
+    K = code.numel()
+    nb = (n + blocksize - 1) // blocksize
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=A.device)
+    if out is None:
+        out = torch.empty(n if K == 256 else (n + 1) // 2, dtype=torch.uint8, device=A.device)
+    _check(lib().bnbq_quantize_blockwise(_dev(code, "code"), K, _dev(A, "A") if n else None, _dtype_id(A), n,
+                                         blocksize, _dev(absmax, "absmax") if n else None,
+                                         _dev(out, "out") if n else None, _stream(stream)))
+    return absmax, out
+
+
+def bnbq_dequantize_blockwise(code: torch.Tensor, q: torch.Tensor, absmax: torch.Tensor, n: int,
+                              blocksize: int = 2048, out_dtype=torch.float32,
+                              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(n, dtype=out_dtype, device=q.device)
+    _check(lib().bnbq_dequantize_blockwise(_dev(code, "code"), code.numel(), _dev(q, "q") if n else None,
+                                           _dev(absmax, "absmax") if n else None, n, blocksize,
+                                           _dev(out, "out") if n else None, _dtype_id(out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------------------- optimizer step
+@dataclass
+class TensorState:
+    """One parameter tensor and its optimizer state (device tensors, contiguous)."""
+    p: torch.Tensor                   # float32
+    g: torch.Tensor                   # float32 or bfloat16
+    state1: torch.Tensor              # uint8 (8-bit) or float32 (32-bit)
+    state2: Optional[torch.Tensor] = None
+    absmax1: Optional[torch.Tensor] = None
+    absmax2: Optional[torch.Tensor] = None
+
+    @property
+    def state_bits(self) -> int:
+        return 8 if self.state1.dtype == torch.uint8 else 32
+
+
+def pack_tensor_list(tensors: Sequence[TensorState]):
+    arr = (CTensor * max(1, len(tensors)))()
+    for i, t in enumerate(tensors):
+        if t.p.dtype != torch.float32:
+            raise TypeError("parameters must be float32")
+        c = arr[i]
+        c.p = _dev(t.p, "p")
+        c.g = _dev(t.g, "g")
+        c.state1 = _dev(t.state1, "state1")
+        c.state2 = _dev(t.state2, "state2") if t.state2 is not None else None
+        c.absmax1 = _dev(t.absmax1, "absmax1") if t.absmax1 is not None else None
+        c.absmax2 = _dev(t.absmax2, "absmax2") if t.absmax2 is not None else None
+        c.n = t.p.numel()
+        c.g_dtype = _dtype_id(t.g)
+        c.state_bits = t.state_bits
+    return arr
+
+
+def bnbq_step_8bit(opt: str | int, tensors: Sequence[TensorState] | ctypes.Array, *, lr: float, beta1: float,
+                   beta2: float, eps: float, weight_decay: float, step: int,
+                   code1: Optional[torch.Tensor], code2: Optional[torch.Tensor], blocksize: int = 2048,
+                   stream=None, ntensors: Optional[int] = None) -> None:
+    """One fused optimizer step over the list (one kernel launch).  ``tensors`` may be a list of
+    TensorState or an array already packed by ``pack_tensor_list`` (then give ``ntensors``)."""
+    o = OPTIMS[opt] if isinstance(opt, str) else int(opt)
+    if isinstance(tensors, ctypes.Array):
+        arr, nt = tensors, ntensors
+    else:
+        arr, nt = pack_tensor_list(tensors), len(tensors)
+    hp = CHParams(lr, beta1, beta2, eps, weight_decay)
+    _check(lib().bnbq_step_8bit(o, arr, nt, ctypes.byref(hp), step,
+                                code1.data_ptr() if code1 is not None else None,
+                                code2.data_ptr() if code2 is not None else None, blocksize, _stream(stream)))
+
+
+def bnbq_device_flags(clear: bool = False) -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib().bnbq_device_flags(ctypes.byref(v), int(clear)))
+    return int(v.value)
+
+
+def bnbq_release() -> None:
+    lib().bnbq_release()
+
+
+def bnbq_version() -> str:
+    return lib().bnbq_version().decode()
+
+
+def bnbq_last_error() -> str:
+    return lib().bnbq_last_error().decode()

@@ -1,0 +1,60 @@
+// bnbq_internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bnbq.h"
+
+namespace bnbq {
+
+// Set the thread-local error text and return `st` (printf-style).
+bnbq_status fail(bnbq_status st, const char* fmt, ...);
+// Map a CUDA error to BNBQ_ECUDA with its text (cudaSuccess -> BNBQ_OK).
+bnbq_status cuda_status(cudaError_t e, const char* what);
+
+// Device-side flag word of the current device (a __device__ variable; its address is taken
+// once per device).
+bnbq_status device_flag_ptr(unsigned** out);
+
+// Number of SMs of the current device (cached per device).
+bnbq_status sm_count(int* out);
+
+// Kernel launchers (argument checks already done by the caller).
+bnbq_status launch_quantize(const float* code, int K, const void* A, bnbq_dtype dt, int64_t n,
+                            int B, float* absmax, uint8_t* out, cudaStream_t s);
+bnbq_status launch_dequantize(const float* code, int K, const uint8_t* q, const float* absmax,
+                              int64_t n, int B, void* out, bnbq_dtype dt, cudaStream_t s);
+
+// One entry of the device descriptor table used by the step kernel (64 bytes).
+struct alignas(16) StepDesc {
+    float* p;
+    const void* g;
+    void* s1;
+    void* s2;
+    float* a1;
+    float* a2;
+    int64_t n;
+    int32_t first_block;  // global index of this tensor's first block
+    int32_t flags;        // bit 0: g is bf16; bit 1: 8-bit state
+};
+static_assert(sizeof(StepDesc) == 64, "descriptor layout");
+constexpr int32_t kDescGBf16 = 1;
+constexpr int32_t kDescState8 = 2;
+
+// Scalars of one step, derived on the host (double, rounded once to binary32).
+struct StepScalars {
+    float b1, b2, omb1, omb2;
+    float step_size;     // lr / (1 - b1^t)
+    float sqrt_bc2;      // sqrt(1 - b2^t)
+    float rcp_sqrt_bc2;  // RN(1 / sqrt_bc2)
+    float decay;         // 1 - lr*wd (AdamW, Lion) or 1
+    float lr, eps, wd;
+    int bc2_fast;        // sqrt_bc2 inside the FMA-quotient range
+};
+
+bnbq_status launch_step(bnbq_optim opt, const StepDesc* d_table, int ntensors, int total_blocks,
+                        const StepScalars& sc, const float* code1, const float* code2, int B,
+                        cudaStream_t s);
+
+}  // namespace bnbq

@@ -1,0 +1,333 @@
+// bnbq_quant.cu -- standalone block-wise quantize / dequantize kernels for sm_100a.
+//
+// Block-wise quantization ("8-bit Optimizers via Block-wise Quantization", abstract, quoted on
+// the blog.csdn.net bitsandbytes guide, section 2): blocks of B consecutive elements are
+// scaled by their own absolute maximum and quantized independently; here one group of B/16
+// threads owns one block (16 elements per thread, as four 4-element chunks whose addresses are
+// consecutive across the group, so every load and store is a fully coalesced vector access).
+// NF4 packing (two 4-bit codes per byte) follows the 4-bit type of the page "Bitsandbytes",
+// section "Normal Float 4 (NF4)".
+//
+// Roofline: HBM.  Quantize moves 4 (fp32) or 2 (bf16) bytes in and 1 (8-bit) or 0.5 (NF4)
+// bytes out per element, plus 4 bytes per block; dequantize the reverse.  The grid is
+// persistent: SMs x resident CTAs, each CTA striding over blocks.
+#include <float.h>
+
+#include "bnbq_device.cuh"
+#include "bnbq_internal.h"
+
+namespace bnbq {
+namespace {
+
+constexpr int kEPT = 16;  // elements per thread per block
+
+template <int B>
+struct QGeom {
+    static constexpr int G = B / kEPT;                   // threads per block-group
+    static constexpr int kThreads = G < 128 ? 128 : G;   // CTA size
+    static constexpr int kGroups = kThreads / G;         // block-groups per CTA
+    static constexpr int kWarps = kThreads / 32;
+};
+
+template <bool BF16>
+__device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, float (&v)[4])
+{
+    if (e + 4 <= n) {
+        if (BF16) {
+            uint2 w = ld_stream_u2(static_cast<const uint16_t*>(A) + e);
+            v[0] = bf16lo_to_f32(w.x);
+            v[1] = bf16hi_to_f32(w.x);
+            v[2] = bf16lo_to_f32(w.y);
+            v[3] = bf16hi_to_f32(w.y);
+        } else {
+            float4 f = ld_stream_f4(static_cast<const float*>(A) + e);
+            v[0] = f.x;
+            v[1] = f.y;
+            v[2] = f.z;
+            v[3] = f.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            float x = 0.0f;
+            if (e + i < n) {
+                if (BF16)
+                    x = __uint_as_float((uint32_t)(static_cast<const uint16_t*>(A)[e + i]) << 16);
+                else
+                    x = static_cast<const float*>(A)[e + i];
+            }
+            v[i] = x;
+        }
+    }
+}
+
+// Stage a codebook in shared memory; returns false (and raises the flag once) if it is invalid.
+__device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with_table, bool& tiny,
+                               unsigned* flags)
+{
+    stage_code_pass1(cs, code, K);
+    __syncthreads();
+    bool bad = false, t = false;
+    stage_code_pass2(cs, K, bad, t);
+    bad = __syncthreads_or(bad);
+    tiny = __syncthreads_or(t);
+    if (bad) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
+        return false;
+    }
+    if (with_table) {
+        stage_code_pass3(cs, K);
+        __syncthreads();
+    }
+    return true;
+}
+
+template <int B, bool BF16, int K>
+__global__ void __launch_bounds__(QGeom<B>::kThreads)
+quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
+                float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags)
+{
+    using Geo = QGeom<B>;
+    constexpr int G = Geo::G;
+    __shared__ CodeSmem cs;
+    __shared__ float red[2][Geo::kWarps];
+
+    bool tiny;
+    if (!stage_one_code(cs, code, K, true, tiny, flags)) return;
+
+    const int gi = threadIdx.x / G;
+    const int tg = threadIdx.x % G;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
+    const int64_t nb = (n + B - 1) / B;
+    int parity = 0;
+
+    for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb;
+         b += (int64_t)gridDim.x * Geo::kGroups) {
+        const int64_t base = b * B;
+        float v[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) load_chunk<BF16>(A, base + 4 * (j * G + tg), n, v[j]);
+
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) m = max_nan(m, fabsf(v[j][i]));
+
+        if constexpr (G <= 32) {
+            m = group_max_nan<G>(m, gmask);
+        } else {
+            m = group_max_nan<32>(m, 0xffffffffu);
+            if (lane == 0) red[parity][warp] = m;
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < Geo::kWarps; w++) m = max_nan(m, red[parity][w]);
+            parity ^= 1;
+        }
+        if (tg == 0) {
+            absmax[b] = m;
+            if (!(m <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
+        }
+        const BlockScale sc = make_scale(m, !tiny);
+
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int64_t e = base + 4 * (j * G + tg);
+            if (e >= n) continue;
+            uint32_t q[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) q[i] = nearest_code(cs, normalise(v[j][i], sc));
+            if constexpr (K == 256) {
+                if (e + 4 <= n) {
+                    st_stream_u32(out + e, q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24));
+                } else {
+                    for (int i = 0; i < 4; i++)
+                        if (e + i < n) out[e + i] = (uint8_t)q[i];
+                }
+            } else {  // two 4-bit codes per byte, even element in the high nibble
+                uint8_t b0 = (uint8_t)((q[0] << 4) | (e + 1 < n ? q[1] : 0u));
+                uint8_t b1 = (uint8_t)((q[2] << 4) | (e + 3 < n ? q[3] : 0u));
+                uint8_t* o = out + (e >> 1);
+                if (e + 4 <= n) {
+                    *reinterpret_cast<uint16_t*>(o) = (uint16_t)(b0 | (b1 << 8));
+                } else {
+                    o[0] = b0;
+                    if (e + 2 < n) o[1] = b1;
+                }
+            }
+        }
+    }
+}
+
+// Dequantize: flat grid over 4-element chunks; each thread takes 4 chunks per pass.
+template <int K, bool BF16OUT>
+__global__ void __launch_bounds__(256)
+dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
+                  const float* __restrict__ absmax, int64_t n, int log2B, void* __restrict__ out,
+                  unsigned* flags)
+{
+    __shared__ CodeSmem cs;
+    bool tiny;
+    if (!stage_one_code(cs, code, K, false, tiny, flags)) return;
+
+    const int64_t nchunks = (n + 3) / 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < nchunks; c0 += 4 * stride) {
+        uint32_t w[4];
+        float a[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int64_t c = c0 + u * stride;
+            w[u] = 0;
+            a[u] = 0.0f;
+            if (c < nchunks) {
+                const int64_t e = 4 * c;
+                if (K == 256) {
+                    if (e + 4 <= n) {
+                        w[u] = ld_stream_u32(q + e);
+                    } else {
+                        for (int i = 0; i < 4; i++)
+                            if (e + i < n) w[u] |= (uint32_t)q[e + i] << (8 * i);
+                    }
+                } else {
+                    if (e + 4 <= n) {
+                        w[u] = __ldcs(reinterpret_cast<const unsigned short*>(q + (e >> 1)));
+                    } else {
+                        w[u] = q[e >> 1];
+                        if (e + 2 < n) w[u] |= (uint32_t)q[(e >> 1) + 1] << 8;
+                    }
+                }
+                a[u] = __ldg(absmax + (e >> log2B));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int64_t c = c0 + u * stride;
+            if (c >= nchunks) continue;
+            const int64_t e = 4 * c;
+            uint32_t idx[4];
+            if (K == 256) {
+                idx[0] = w[u] & 0xff;
+                idx[1] = (w[u] >> 8) & 0xff;
+                idx[2] = (w[u] >> 16) & 0xff;
+                idx[3] = w[u] >> 24;
+            } else {
+                idx[0] = (w[u] >> 4) & 0xf;
+                idx[1] = w[u] & 0xf;
+                idx[2] = (w[u] >> 12) & 0xf;
+                idx[3] = (w[u] >> 8) & 0xf;
+            }
+            float y[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) y[i] = __fmul_rn(cs.code[idx[i]], a[u]);
+            if (e + 4 <= n) {
+                if (BF16OUT) {
+                    st_stream_u2(static_cast<uint16_t*>(out) + e,
+                                 make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3])));
+                } else {
+                    st_stream_f4(static_cast<float*>(out) + e, make_float4(y[0], y[1], y[2], y[3]));
+                }
+            } else {
+                for (int i = 0; i < 4; i++) {
+                    if (e + i >= n) break;
+                    if (BF16OUT)
+                        static_cast<__nv_bfloat16*>(out)[e + i] = __float2bfloat16_rn(y[i]);
+                    else
+                        static_cast<float*>(out)[e + i] = y[i];
+                }
+            }
+        }
+    }
+}
+
+template <typename Kern>
+bnbq_status persistent_grid(Kern kern, int threads, int64_t work_units, int units_per_cta, int* grid)
+{
+    int sms = 0;
+    bnbq_status st = sm_count(&sms);
+    if (st != BNBQ_OK) return st;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+    if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1) per_sm = 1;
+    int64_t need = (work_units + units_per_cta - 1) / units_per_cta;
+    int64_t g = (int64_t)sms * per_sm;
+    *grid = (int)(need < g ? (need < 1 ? 1 : need) : g);
+    return BNBQ_OK;
+}
+
+template <int B, bool BF16, int K>
+bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax, uint8_t* out,
+                     cudaStream_t s)
+{
+    using Geo = QGeom<B>;
+    unsigned* flags = nullptr;
+    bnbq_status st = device_flag_ptr(&flags);
+    if (st != BNBQ_OK) return st;
+    int grid = 0;
+    auto kern = quantize_kernel<B, BF16, K>;
+    st = persistent_grid(kern, Geo::kThreads, (n + B - 1) / B, Geo::kGroups, &grid);
+    if (st != BNBQ_OK) return st;
+    kern<<<grid, Geo::kThreads, 0, s>>>(code, A, n, absmax, out, flags);
+    return cuda_status(cudaGetLastError(), "quantize_kernel launch");
+}
+
+template <int B, bool BF16>
+bnbq_status launch_q_k(const float* code, int K, const void* A, int64_t n, float* absmax,
+                       uint8_t* out, cudaStream_t s)
+{
+    return K == 256 ? launch_q<B, BF16, 256>(code, A, n, absmax, out, s)
+                    : launch_q<B, BF16, 16>(code, A, n, absmax, out, s);
+}
+
+template <int B>
+bnbq_status launch_q_b(const float* code, int K, const void* A, bnbq_dtype dt, int64_t n,
+                       float* absmax, uint8_t* out, cudaStream_t s)
+{
+    return dt == BNBQ_BF16 ? launch_q_k<B, true>(code, K, A, n, absmax, out, s)
+                           : launch_q_k<B, false>(code, K, A, n, absmax, out, s);
+}
+
+template <int K, bool BF16OUT>
+bnbq_status launch_dq(const float* code, const uint8_t* q, const float* absmax, int64_t n, int B,
+                      void* out, cudaStream_t s)
+{
+    unsigned* flags = nullptr;
+    bnbq_status st = device_flag_ptr(&flags);
+    if (st != BNBQ_OK) return st;
+    int log2B = 0;
+    while ((1 << log2B) < B) log2B++;
+    int grid = 0;
+    auto kern = dequantize_kernel<K, BF16OUT>;
+    st = persistent_grid(kern, 256, (n + 3) / 4, 256 * 4, &grid);
+    if (st != BNBQ_OK) return st;
+    kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags);
+    return cuda_status(cudaGetLastError(), "dequantize_kernel launch");
+}
+
+}  // namespace
+
+bnbq_status launch_quantize(const float* code, int K, const void* A, bnbq_dtype dt, int64_t n,
+                            int B, float* absmax, uint8_t* out, cudaStream_t s)
+{
+    switch (B) {
+        case 256: return launch_q_b<256>(code, K, A, dt, n, absmax, out, s);
+        case 2048: return launch_q_b<2048>(code, K, A, dt, n, absmax, out, s);
+        case 4096: return launch_q_b<4096>(code, K, A, dt, n, absmax, out, s);
+        default: return fail(BNBQ_EINVAL, "blocksize %d not in {256, 2048, 4096}", B);
+    }
+}
+
+bnbq_status launch_dequantize(const float* code, int K, const uint8_t* q, const float* absmax,
+                              int64_t n, int B, void* out, bnbq_dtype dt, cudaStream_t s)
+{
+    if (K == 256)
+        return dt == BNBQ_BF16 ? launch_dq<256, true>(code, q, absmax, n, B, out, s)
+                               : launch_dq<256, false>(code, q, absmax, n, B, out, s);
+    return dt == BNBQ_BF16 ? launch_dq<16, true>(code, q, absmax, n, B, out, s)
+                           : launch_dq<16, false>(code, q, absmax, n, B, out, s);
+}
+
+}  // namespace bnbq

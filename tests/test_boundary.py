@@ -1,0 +1,159 @@
+"""CPU-only checks of the C ABI boundary (no kernel runs here).
+
+* the shared library loads and exports every entry point declared in include/bnbq.h;
+* its host-side codebooks equal the oracle's and the golden fixtures (independent builds);
+* argument checks reject bad input synchronously, before any CUDA call, with a message;
+* the launcher policy (which tensors keep 32-bit state) and the workload shapes.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_wise_bit_b200 import bindings as B
+from block_wise_bit_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bnbq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bnbq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = B.lib()
+    declared = _declared()
+    assert len(declared) >= 10, declared
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared in bnbq.h but not exported"
+    assert set(declared) == set(B.EXPORTED)
+    assert B.bnbq_version() == "0.1.0"
+
+
+def test_only_bnbq_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {B.library_path()}").read().split("\n")
+    funcs = [ln.split()[-1] for ln in out if " T " in ln]
+    assert funcs and all(f.startswith("bnbq_") for f in funcs), funcs
+
+
+@pytest.mark.parametrize("kind", ["dynamic_signed", "dynamic_unsigned", "nf4", "linear"])
+def test_library_codebooks_match_oracle_and_golden(oracle_mod, kind):
+    lib_code = B.bnbq_codebook(kind).numpy()
+    np.testing.assert_array_equal(lib_code, getattr(oracle_mod, "code_" + kind)())
+    path = os.path.join(ROOT, "tests", "golden", f"code_{kind}.hex")
+    gold = [float.fromhex(x.strip()) for x in open(path) if x.strip() and not x.startswith("#")]
+    np.testing.assert_array_equal(lib_code, np.array(gold, np.float32))
+    B.bnbq_check_codebook(B.bnbq_codebook(kind))
+
+
+def test_check_codebook_rejects():
+    import torch
+    good = B.bnbq_codebook("dynamic_signed")
+    for bad in (good.flip(0), torch.cat([good[:-1], torch.tensor([2.0])]),
+                torch.cat([good[:-1], torch.tensor([float("nan")])]), good[:100]):
+        with pytest.raises(B.BnbqError) as e:
+            B.bnbq_check_codebook(bad)
+        assert e.value.status == B.EINVAL and B.bnbq_last_error()
+
+
+def _q(code=0x1000, K=256, A=0x2000, dt=0, n=100, Bs=2048, am=0x3000, out=0x4000):
+    return B.lib().bnbq_quantize_blockwise(code, K, A, dt, n, Bs, am, out, None)
+
+
+def test_quantize_argument_checks():
+    assert _q(code=None) == B.EINVAL
+    assert _q(K=17) == B.EINVAL
+    assert _q(Bs=1024) == B.EINVAL
+    assert _q(n=-1) == B.EINVAL
+    assert _q(dt=7) == B.EINVAL
+    assert _q(A=None) == B.EINVAL
+    assert _q(A=0x2004) == B.EINVAL          # fp32 input must be 16-byte aligned
+    assert _q(out=0x4001) == B.EINVAL
+    assert _q(K=16, out=0x4001) == B.EINVAL
+    assert _q(am=0x3002) == B.EINVAL
+    assert "aligned" in B.bnbq_last_error()
+    assert _q(n=0, A=None, am=None, out=None) == B.OK  # empty: no-op, no CUDA call
+
+
+def test_dequantize_argument_checks():
+    L = B.lib()
+    assert L.bnbq_dequantize_blockwise(0x1000, 256, 0x2000, 0x3000, 10, 100, 0x4000, 0, None) == B.EINVAL
+    assert L.bnbq_dequantize_blockwise(0x1000, 256, 0x2002, 0x3000, 10, 256, 0x4000, 0, None) == B.EINVAL
+    assert L.bnbq_dequantize_blockwise(0x1000, 16, 0x2002, 0x3000, 10, 256, 0x4008, 0, None) == B.EINVAL
+    assert L.bnbq_dequantize_blockwise(0x1000, 256, 0x2000, 0x3000, 10, 256, 0x4000, 5, None) == B.EINVAL
+    assert L.bnbq_dequantize_blockwise(0x1000, 256, None, None, 0, 256, None, 0, None) == B.OK
+
+
+def _t(**kw):
+    d = dict(p=0x10000, g=0x20000, state1=0x30000, state2=0x40000, absmax1=0x50000, absmax2=0x60000, n=5000,
+             g_dtype=1, state_bits=8)
+    d.update(kw)
+    return B.CTensor(**d)
+
+
+def _step(opt=0, tensors=None, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), step=1, c1=0x7000, c2=0x8000, Bs=2048):
+    tensors = [_t()] if tensors is None else tensors
+    arr = (B.CTensor * max(1, len(tensors)))(*tensors)
+    h = B.CHParams(*hp)
+    return B.lib().bnbq_step_8bit(opt, arr, len(tensors), ctypes.byref(h), step, c1, c2, Bs, None)
+
+
+def test_step_argument_checks():
+    assert _step(opt=9) == B.EINVAL
+    assert _step(step=0) == B.EINVAL
+    assert _step(Bs=512) == B.EINVAL
+    assert _step(hp=(1e-3, 1.0, 0.999, 1e-8, 0.0)) == B.EINVAL   # Adam beta1 must be < 1
+    assert _step(hp=(float("nan"), 0.9, 0.999, 1e-8, 0.0)) == B.EINVAL
+    assert _step(tensors=[_t(n=-5)]) == B.EINVAL
+    assert _step(tensors=[_t(state_bits=16)]) == B.EINVAL
+    assert _step(tensors=[_t(g_dtype=3)]) == B.EINVAL
+    assert _step(tensors=[_t(p=0x10004)]) == B.EINVAL
+    assert _step(tensors=[_t(g=0x20004)]) == B.EINVAL           # bf16 needs 8-byte alignment
+    assert _step(tensors=[_t(state1=0x30002)]) == B.EINVAL
+    assert _step(tensors=[_t(state_bits=32, state1=0x30008)]) == B.EINVAL
+    assert _step(tensors=[_t(absmax2=None)]) == B.EINVAL
+    assert _step(tensors=[_t(state2=None)]) == B.EINVAL
+    assert _step(c2=None) == B.EINVAL                           # Adam 8-bit needs the unsigned code
+    assert "code" in B.bnbq_last_error()
+    # empty entries and empty lists are no-ops (no CUDA call)
+    assert _step(tensors=[_t(n=0)]) == B.OK
+    assert _step(tensors=[]) == B.OK
+    # one-state optimizers ignore state2 / absmax2 / code2
+    assert _step(opt=2, tensors=[_t(n=-1)]) == B.EINVAL
+    h = B.CHParams(1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert B.lib().bnbq_step_8bit(0, None, 3, ctypes.byref(h), 1, 0x7000, 0x8000, 2048, None) == B.EINVAL
+    assert B.lib().bnbq_step_8bit(0, None, 0, None, 1, 0x7000, 0x8000, 2048, None) == B.EINVAL
+
+
+def test_state_policy_and_shapes():
+    assert W.state_bits_for(W.ParamSpec("a", 4095)) == 32
+    assert W.state_bits_for(W.ParamSpec("a", 4096)) == 8       # "fewer than 4096" is strict
+    assert W.state_bits_for(W.ParamSpec("e", 10 ** 8, embedding=True)) == 32
+    assert W.state_bits_for(W.ParamSpec("a", 10000), min_8bit_size=16384) == 32
+    g = W.gpt2_1p5b()
+    assert len(g) == 580 and sum(s.numel for s in g) == 1_557_611_200
+    lay = W.Layout.build(g, 2048)
+    assert lay.state_bits.count(32) == 291 and lay.n32 == 80_875_200
+    assert sum(1 for s, b in zip(g, lay.state_bits) if b == 8 and s.numel % 2048) == 96
+    ll = W.llama7b()
+    assert len(ll) == 291 and sum(s.numel for s in ll) == 6_738_415_616
+    lay = W.Layout.build(ll, 2048)
+    assert lay.state_bits.count(32) == 1 and lay.n32 == 131_072_000
+    assert lay.n8 == 6_607_343_616 and lay.n_blocks8 == 3_226_242
+    assert sum(s.numel for s in W.llama7b_layer()) == 202_383_360
+    # every flat offset keeps 16-byte alignment for fp32 and 4-byte alignment for codes
+    assert all(o % 4 == 0 for o in lay.off + [x for x in lay.off8 if x >= 0] + [x for x in lay.off32 if x >= 0])
+
+
+def test_algorithmic_bytes_model():
+    """Bytes per step of the 7B AdamW list: 14 B per 8-bit-state param (bf16 grads), 26 B per
+    32-bit-state param, 16 B per block of scales."""
+    from bench import algorithmic_bytes
+    lay = W.Layout.build(W.llama7b(), 2048)
+    assert algorithmic_bytes(lay, "adamw", g_bytes=2) == 6_607_343_616 * 14 + 3_226_242 * 16 + 131_072_000 * 26
+    assert algorithmic_bytes(lay, "lion", g_bytes=2) == 6_607_343_616 * 12 + 3_226_242 * 8 + 131_072_000 * 18

@@ -1,0 +1,305 @@
+"""GPU parity: the fused multi-tensor optimizer step through the C ABI against the CPU oracle.
+
+* Tiny 8-bit AdamW: one 65,536-element fp32 tensor ~N(0,0.02), fp32 grads ~N(0,1e-3) drawn
+  afresh each step (seed 0), blocksize 2048, zero initial state, lr 1e-3, betas (0.9, 0.999),
+  eps 1e-8, wd 0.01, 10 steps: GPU and oracle each run their own trajectory; compared at every
+  step.  Plus standalone quantize / dequantize of the same tensor.
+* Every optimizer x blocksize x gradient dtype on a small multi-tensor list with ragged tails
+  and 32-bit-state members, from a synthetic non-zero state, several steps.
+* GPT-2-1.5B AdamW and 7B Llama AdamW / Lion / momentum lists at full size, stepped whole by
+  one launch per step (the benchmark's launch configuration); sampled tensors / block ranges are
+  recomputed by the oracle from the same seeded inputs along their own trajectory.
+Bar: p within 1e-6 relative or 1e-9 absolute; codes equal except within 2 ulp of a decision
+boundary (fraction < 1e-5); absmax mismatches reported (expected: none, fully bit-exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_wise_bit_b200 as bq
+from block_wise_bit_b200 import optim as O
+from block_wise_bit_b200 import workloads as W
+
+from . import parity
+import oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+HP = {
+    "adamw": dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
+    "adam": dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
+    "lion": dict(lr=1e-4, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=0.1),
+    "momentum": dict(lr=1e-2, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=0.0),
+}
+REPORT = []
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    bq.lib()
+    bq.bnbq_device_flags(clear=True)
+    yield
+    assert bq.bnbq_device_flags(clear=True) == 0
+    for line in REPORT:
+        print(line)
+
+
+def _codes():
+    return bq.bnbq_codebook("dynamic_signed"), bq.bnbq_codebook("dynamic_unsigned")
+
+
+class HostTensor:
+    """Host (numpy) copy of one tensor's step inputs, advanced by the oracle."""
+
+    def __init__(self, ts: bq.TensorState):
+        self.p = parity.to_np(ts.p)
+        self.s1 = parity.to_np(ts.state1)
+        self.s2 = parity.to_np(ts.state2) if ts.state2 is not None else None
+        self.a1 = parity.to_np(ts.absmax1) if ts.absmax1 is not None else None
+        self.a2 = parity.to_np(ts.absmax2) if ts.absmax2 is not None else None
+
+
+def _compare(name, ts, ht, g_np, optim, B, t, c1, c2, prev):
+    """Compare GPU tensor ``ts`` with host copy ``ht`` after both stepped; ``prev`` is the
+    pre-step host state (for classifying code mismatches)."""
+    n_pdiff = parity.assert_p_close(parity.to_np(ts.p), ht.p, f"{name} t={t} p")
+    if ht.s1.dtype == np.uint8:
+        m1, v1 = parity.oracle_new_moments(optim, prev.p, g_np, prev.s1, prev.s2, prev.a1, prev.a2, c1, c2, B,
+                                           HP[optim], t)
+        n1, am1 = parity.compare_state(parity.to_np(ts.state1), ht.s1, parity.to_np(ts.absmax1), ht.a1, c1,
+                                       parity.blockwise_normalised(m1, ht.a1, B), f"{name} t={t} state1")
+        n2 = am2 = 0
+        if ht.s2 is not None:
+            n2, am2 = parity.compare_state(parity.to_np(ts.state2), ht.s2, parity.to_np(ts.absmax2), ht.a2, c2,
+                                           parity.blockwise_normalised(v1, ht.a2, B), f"{name} t={t} state2")
+        REPORT.append(f"{name} t={t}: p bit-diff {n_pdiff}, code mismatches {n1}+{n2}, absmax mismatches {am1}+{am2}")
+        return n_pdiff + n1 + n2 + am1 + am2
+    s1 = parity.to_np(ts.state1)
+    np.testing.assert_allclose(s1, ht.s1, rtol=1e-6, atol=1e-12)
+    nd = int(np.count_nonzero(s1.view(np.uint32) != ht.s1.view(np.uint32)))
+    if ht.s2 is not None:
+        s2 = parity.to_np(ts.state2)
+        np.testing.assert_allclose(s2, ht.s2, rtol=1e-6, atol=1e-18)
+        nd += int(np.count_nonzero(s2.view(np.uint32) != ht.s2.view(np.uint32)))
+    REPORT.append(f"{name} t={t}: p bit-diff {n_pdiff}, 32-bit state bit-diff {nd}")
+    return n_pdiff + nd
+
+
+def _copy_prev(ht):
+    prev = HostTensor.__new__(HostTensor)
+    for k in ("p", "s1", "s2", "a1", "a2"):
+        v = getattr(ht, k)
+        setattr(prev, k, None if v is None else v.copy())
+    return prev
+
+
+def test_tiny_adamw_trajectory_and_quantize():
+    n, B, optim = 65536, 2048, "adamw"
+    c1, c2 = _codes()
+    p = W.normal(n, 0.02, DEV, "tiny", 0, "p")
+    # standalone quantize / dequantize of the same tensor
+    a, q = bq.bnbq_quantize_blockwise(c1.to(DEV), p, B)
+    a_or, q_or = oracle.quantize_blockwise(c1.numpy(), parity.to_np(p), B)
+    np.testing.assert_array_equal(parity.to_np(a).view(np.uint32), a_or.view(np.uint32))
+    np.testing.assert_array_equal(parity.to_np(q), q_or)
+    y = bq.bnbq_dequantize_blockwise(c1.to(DEV), q, a, n, B)
+    np.testing.assert_array_equal(parity.to_np(y).view(np.uint32),
+                                  oracle.dequantize_blockwise(c1.numpy(), q_or, a_or, n, B).view(np.uint32))
+
+    st = O.new_state(p, True, 8, B, c1, c2)
+    g = torch.empty(n, device=DEV)
+    ts = bq.TensorState(p, g, st["state1"], st["state2"], st["absmax1"], st["absmax2"])
+    ht = HostTensor(ts)
+    total = 0
+    for t in range(1, 11):
+        g.copy_(W.normal(n, 1e-3, DEV, "tiny", 0, "g", t))
+        g_np = parity.to_np(g)
+        prev = _copy_prev(ht)
+        bq.bnbq_step_8bit(optim, [ts], step=t, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP[optim])
+        torch.cuda.synchronize()
+        parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(), c2.numpy(), B,
+                                 HP[optim], t)
+        total += _compare("tiny", ts, ht, g_np, optim, B, t, c1.numpy(), c2.numpy(), prev)
+    REPORT.append(f"tiny AdamW 10-step trajectory: total differing elements {total}")
+
+
+SIZES = [1, 3, 5, 4095, 4096, 4100, 2048 * 3 + 17, 65536, 70001]
+
+
+def _small_list(optim, B, g_dtype, seed):
+    """Tensors of SIZES (policy: < 4096 -> 32-bit) plus one large tensor forced to 32-bit, with
+    a synthetic non-zero state."""
+    two = optim in ("adamw", "adam")
+    c1, c2 = _codes()
+    out = []
+    for i, n in enumerate(SIZES + [30000]):
+        bits = 32 if (n < 4096 or i == len(SIZES)) else 8
+        p = W.normal(n, 0.02, DEV, "small", seed, i, "p")
+        g = W.normal(n, 1e-3, DEV, "small", seed, i, "g").to(g_dtype)
+        if bits == 8:
+            nb = (n + B - 1) // B
+            s1 = W.random_codes(n, DEV, "small", seed, i, "q1")
+            a1 = W.log_uniform(nb, 1e-4, 1e-2, DEV, "small", seed, i, "a1")
+            s2 = W.random_codes(n, DEV, "small", seed, i, "q2") if two else None
+            a2 = W.log_uniform(nb, 1e-8, 1e-5, DEV, "small", seed, i, "a2") if two else None
+            if optim == "momentum":
+                a1 = W.log_uniform(nb, 1e-3, 1e-1, DEV, "small", seed, i, "a1m")
+        else:
+            s1 = W.normal(n, 1e-3, DEV, "small", seed, i, "m")
+            s2 = W.normal(n, 1e-3, DEV, "small", seed, i, "v").square_() if two else None
+            a1 = a2 = None
+        out.append(bq.TensorState(p, g, s1, s2, a1, a2))
+    return out, c1, c2
+
+
+@pytest.mark.parametrize("optim", ["adamw", "adam", "lion", "momentum"])
+@pytest.mark.parametrize("B", [256, 2048, 4096])
+@pytest.mark.parametrize("g_dtype", [torch.float32, torch.bfloat16])
+def test_small_list_all_optimizers(optim, B, g_dtype):
+    seed = W.seed_of(optim, B, str(g_dtype)) % 1000
+    tensors, c1, c2 = _small_list(optim, B, g_dtype, seed)
+    hts = [HostTensor(ts) for ts in tensors]
+    two = optim in ("adamw", "adam")
+    for t in (1, 2, 7):
+        prevs = [_copy_prev(h) for h in hts]
+        bq.bnbq_step_8bit(optim, tensors, step=t, code1=c1.to(DEV), code2=c2.to(DEV) if two else None, blocksize=B,
+                          **HP[optim])
+        torch.cuda.synchronize()
+        for i, (ts, ht, prev) in enumerate(zip(tensors, hts, prevs)):
+            g_np = parity.to_np(ts.g)
+            parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(),
+                                     c2.numpy() if two else None, B, HP[optim], t)
+            _compare(f"{optim}/B{B}/{g_dtype}/#{i}(n={ts.p.numel()})", ts, ht, g_np, optim, B, t, c1.numpy(),
+                     c2.numpy() if two else None, prev)
+
+
+def test_zero_gradient_zero_state_stays_zero():
+    c1, c2 = _codes()
+    n, B = 10000, 2048
+    p = torch.ones(n, device=DEV)
+    st = O.new_state(p, True, 8, B, c1, c2)
+    g = torch.zeros(n, device=DEV)
+    ts = bq.TensorState(p, g, st["state1"], st["state2"], st["absmax1"], st["absmax2"])
+    bq.bnbq_step_8bit("adamw", [ts], step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B,
+                      lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0)
+    assert bool((st["state1"] == 127).all()) and bool((st["state2"] == 0).all())
+    assert bool((st["absmax1"] == 0).all()) and bool((p == 1).all())
+
+
+def test_optimizer_front_end_matches_direct_call():
+    """AdamW8bit over torch parameters (policy: < 4096 elements -> 32-bit; override -> 32-bit)
+    gives the same result as the oracle on each tensor."""
+    c1, c2 = _codes()
+    params = [torch.nn.Parameter(W.normal(n, 0.02, DEV, "fe", i)) for i, n in enumerate([100, 5000, 40000])]
+    opt = O.AdamW8bit(params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.01)
+    opt.override_32bit(params[2])
+    host = []
+    for t in (1, 2):
+        for i, p in enumerate(params):
+            p.grad = W.normal(p.numel(), 1e-3, DEV, "fe-g", i, t)
+        if t == 1:
+            host = [dict(p=parity.to_np(p), bits=opt.state_bits_for(p)) for p in params]
+            for h, p in zip(host, params):
+                n = p.numel()
+                if h["bits"] == 8:
+                    nb = (n + 2047) // 2048
+                    h.update(s1=np.full(n, 127, np.uint8), s2=np.zeros(n, np.uint8), a1=np.zeros(nb, np.float32),
+                             a2=np.zeros(nb, np.float32))
+                else:
+                    h.update(s1=np.zeros(n, np.float32), s2=np.zeros(n, np.float32), a1=None, a2=None)
+        opt.step()
+        torch.cuda.synchronize()
+        for h, p in zip(host, params):
+            parity.oracle_step_numpy("adamw", h["p"], parity.to_np(p.grad), h["s1"], h["s2"], h["a1"], h["a2"],
+                                     c1.numpy(), c2.numpy(), 2048, HP["adamw"], t)
+            parity.assert_p_close(parity.to_np(p.detach()), h["p"], "front-end p")
+    assert [opt.state_bits_for(p) for p in params] == [32, 8, 32]
+
+
+# ---------------------------------------------------------------------------------- full size
+def _sample_ranges(lay, B, picks):
+    """(tensor index, first block, last block) ranges to check: whole small tensors, and for big
+    ones the first 24 blocks plus the final (possibly partial) block."""
+    out = []
+    for i in picks:
+        n = lay.specs[i].numel
+        nb = (n + B - 1) // B
+        if nb <= 32:
+            out.append((i, 0, nb))
+        else:
+            out.append((i, 0, 24))
+            out.append((i, nb - 1, nb))
+    return out
+
+
+def _slice_state(fl, i, b0, b1):
+    """TensorState views of blocks [b0, b1) of tensor i of a FlatStateList."""
+    ts = fl.entries[i]
+    B = fl.layout.blocksize
+    n = ts.p.numel()
+    e0, e1 = b0 * B, min(n, b1 * B)
+    s = lambda x: None if x is None else x[e0:e1]  # noqa: E731
+    a = lambda x: None if x is None else x[b0:b1]  # noqa: E731
+    if ts.absmax1 is not None:
+        return bq.TensorState(ts.p[e0:e1], ts.g[e0:e1], s(ts.state1), s(ts.state2), a(ts.absmax1), a(ts.absmax2))
+    return bq.TensorState(ts.p[e0:e1], ts.g[e0:e1], s(ts.state1), s(ts.state2))
+
+
+def _full_size_run(shape, optim, seed, steps, picks_fn, g_outlier=(0.0, 1.0)):
+    if torch.cuda.get_device_properties(0).total_memory < 80e9 and shape == "llama7b":
+        pytest.skip("needs a GPU with >= 80 GB")
+    B = 2048
+    lay = W.Layout.build(W.SHAPES[shape](), B)
+    fl = O.FlatStateList(lay, optim, DEV, g_dtype=torch.bfloat16)
+    for i, spec in enumerate(lay.specs):
+        fl.entries[i].p.copy_(W.normal(spec.numel, 0.02, DEV, shape, seed, i, "p"))
+    c1, c2 = _codes()
+    two = optim in ("adamw", "adam")
+    ranges = _sample_ranges(lay, B, picks_fn(lay))
+    hosts = [HostTensor(_slice_state(fl, i, b0, b1)) for (i, b0, b1) in ranges]
+    for t in range(1, steps + 1):
+        for i, spec in enumerate(lay.specs):
+            W.grad_fill_(fl.entries[i].g, 1e-3, g_outlier[0], g_outlier[1], shape, seed, i, "g", t)
+        prevs = [_copy_prev(h) for h in hosts]
+        fl.step(t, **HP[optim])
+        torch.cuda.synchronize()
+        for (i, b0, b1), ht, prev in zip(ranges, hosts, prevs):
+            ts = _slice_state(fl, i, b0, b1)
+            g_np = parity.to_np(ts.g)
+            parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(),
+                                     c2.numpy() if two else None, B, HP[optim], t)
+            _compare(f"{shape}/{optim}/{lay.specs[i].name}[{b0}:{b1}]", ts, ht, g_np, optim, B, t, c1.numpy(),
+                     c2.numpy() if two else None, prev)
+    # property over the whole list: every 8-bit block scale is finite and non-negative
+    assert bool(torch.isfinite(fl.a1).all()) and bool((fl.a1 >= 0).all())
+    del fl
+    torch.cuda.empty_cache()
+
+
+def _gpt2_picks(lay):
+    names = [s.name for s in lay.specs]
+    want = ["wte", "wpe", "h0.ln_1.w", "h0.attn.c_attn.w", "h0.attn.c_attn.b", "h0.attn.c_proj.b", "h0.mlp.c_fc.w",
+            "h0.mlp.c_fc.b", "h47.mlp.c_proj.w", "h47.mlp.c_proj.b", "ln_f.b"]
+    return [names.index(w) for w in want]
+
+
+def _llama_picks(lay):
+    names = [s.name for s in lay.specs]
+    want = ["embed_tokens", "layers.0.q_proj", "layers.0.down_proj", "layers.0.input_layernorm",
+            "layers.31.up_proj", "norm", "lm_head"]
+    return [names.index(w) for w in want]
+
+
+def test_gpt2_1p5b_adamw_full_size():
+    _full_size_run("gpt2_1p5b", "adamw", 2, 6, _gpt2_picks)
+
+
+@pytest.mark.parametrize("optim", ["lion", "momentum"])
+def test_llama7b_lion_momentum_full_size(optim):
+    _full_size_run("llama7b", optim, 3, 2, _llama_picks, g_outlier=(1e-4, 100.0))
+
+
+def test_llama7b_adamw_full_size():
+    _full_size_run("llama7b", "adamw", 4, 2, _llama_picks)
