@@ -57,11 +57,12 @@ def library_path() -> str:
 
 
 def lib(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load libbnbq.so (building it with nvcc first if it is missing or stale and nvcc exists)."""
+    """Load libbnbq.so (building it with nvcc first if it is missing or stale and nvcc exists).
+    The environment variable BNBQ_LIBRARY names another build of the same library to load."""
     global _lib
     if _lib is None:
-        path = _build.LIB
-        if build_if_missing:
+        path = os.environ.get("BNBQ_LIBRARY") or _build.LIB
+        if build_if_missing and not os.environ.get("BNBQ_LIBRARY"):
             try:
                 path = _build.build()
             except RuntimeError:

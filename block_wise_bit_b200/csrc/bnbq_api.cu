@@ -456,7 +456,10 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
     if (two && !(sc.sqrt_bc2 > 0.0f)) return fail(BNBQ_EINVAL, "1 - beta2^step rounds to zero");
     volatile float one = 1.0f;  // keep the reciprocal a binary32 division
     sc.rcp_sqrt_bc2 = one / sc.sqrt_bc2;
-    sc.bc2_fast = (sc.sqrt_bc2 >= 0x1p-60f && sc.sqrt_bc2 <= 0x1p100f) ? 1 : 0;
+    // The kernel divides by sqrt(1-b2^t) with the FMA quotient, exact for divisors in
+    // [2^-60, 2^100]; any binary32 beta2 < 1 gives sqrt(1-b2^t) >= 2^-12.
+    if (two && !(sc.sqrt_bc2 >= 0x1p-60f && sc.sqrt_bc2 <= 1.0f))
+        return fail(BNBQ_EINVAL, "sqrt(1 - beta2^step) = %g outside [2^-60, 1]", (double)sc.sqrt_bc2);
     sc.decay = (opt == BNBQ_ADAMW || opt == BNBQ_LION)
                    ? (float)(1.0 - (double)hp->lr * (double)hp->weight_decay)
                    : 1.0f;

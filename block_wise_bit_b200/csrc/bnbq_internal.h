@@ -50,7 +50,6 @@ struct StepScalars {
     float rcp_sqrt_bc2;  // RN(1 / sqrt_bc2)
     float decay;         // 1 - lr*wd (AdamW, Lion) or 1
     float lr, eps, wd;
-    int bc2_fast;        // sqrt_bc2 inside the FMA-quotient range
 };
 
 bnbq_status launch_step(bnbq_optim opt, const StepDesc* d_table, int ntensors, int total_blocks,

@@ -21,14 +21,15 @@ namespace {
 
 constexpr int kEPT = 16;  // elements per thread per block
 
+constexpr int kQThreads = 512;
+
 template <int B>
 struct QGeom {
-    static constexpr int G = B / kEPT;                   // threads per block-group
-    static constexpr int kThreads = G < 128 ? 128 : G;   // CTA size
-    static constexpr int kGroups = kThreads / G;         // block-groups per CTA
-    static constexpr int kWarps = kThreads / 32;
+    static constexpr int G = B / kEPT;                 // threads per block-group
+    static constexpr int kGroups = kQThreads / G;      // block-groups per CTA
+    static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
+    static constexpr size_t kSmem = sizeof(CodeSmem) + sizeof(float) * kGroups * 2 * kGroupWarps;
 };
-
 template <bool BF16>
 __device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, float (&v)[4])
 {
@@ -61,50 +62,42 @@ __device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, 
     }
 }
 
-// Stage a codebook in shared memory; returns false (and raises the flag once) if it is invalid.
-__device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with_table, bool& tiny,
-                               unsigned* flags)
+// Stage the codes (and, with_table, midpoints and bucket table) in shared memory.  Returns
+// false, raising the flag once, if the codebook is invalid; `fast` = FMA quotient allowed;
+// `general` = some bucket needs the general search.
+__device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with_table, bool& fast,
+                               bool& general, unsigned* flags)
 {
     stage_code_pass1(cs, code, K);
     __syncthreads();
     bool bad = false, t = false;
     stage_code_pass2(cs, K, bad, t);
     bad = __syncthreads_or(bad);
-    tiny = __syncthreads_or(t);
+    fast = !__syncthreads_or(t);
     if (bad) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
         return false;
     }
-    if (with_table) {
-        stage_code_pass3(cs, K);
-        __syncthreads();
-    }
+    general = false;
+    if (with_table) general = __syncthreads_or(stage_code_pass3(cs, K));
     return true;
 }
 
-template <int B, bool BF16, int K>
-__global__ void __launch_bounds__(QGeom<B>::kThreads)
-quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
-                float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags)
+template <int B, bool BF16, int K, bool GENERAL>
+__device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
+                                              float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
+                                              unsigned* flags)
 {
     using Geo = QGeom<B>;
     constexpr int G = Geo::G;
-    __shared__ CodeSmem cs;
-    __shared__ float red[2][Geo::kWarps];
-
-    bool tiny;
-    if (!stage_one_code(cs, code, K, true, tiny, flags)) return;
-
     const int gi = threadIdx.x / G;
     const int tg = threadIdx.x % G;
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
     const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
     const int64_t nb = (n + B - 1) / B;
     int parity = 0;
 
-    for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb;
-         b += (int64_t)gridDim.x * Geo::kGroups) {
+    for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb; b += (int64_t)gridDim.x * Geo::kGroups) {
         const int64_t base = b * B;
         float v[4][4];
 #pragma unroll
@@ -119,36 +112,40 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
         if constexpr (G <= 32) {
             m = group_max_nan<G>(m, gmask);
         } else {
+            constexpr int W = G / 32;
             m = group_max_nan<32>(m, 0xffffffffu);
-            if (lane == 0) red[parity][warp] = m;
-            __syncthreads();
+            float* r = red + (gi * 2 + parity) * W;
+            if (lane == 0) r[tg >> 5] = m;
+            group_barrier(1 + gi, G);
 #pragma unroll
-            for (int w = 0; w < Geo::kWarps; w++) m = max_nan(m, red[parity][w]);
+            for (int w = 0; w < W; w++) m = max_nan(m, r[w]);
             parity ^= 1;
         }
         if (tg == 0) {
             absmax[b] = m;
             if (!(m <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
         }
-        const BlockScale sc = make_scale(m, !tiny);
+        const BlockScale sc = make_scale(m, fast);
 
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const int64_t e = base + 4 * (j * G + tg);
             if (e >= n) continue;
-            uint32_t q[4];
-#pragma unroll
-            for (int i = 0; i < 4; i++) q[i] = nearest_code(cs, normalise(v[j][i], sc));
+            const float2 x0 = normalise2(make_float2(v[j][0], v[j][1]), sc);
+            const float2 x1 = normalise2(make_float2(v[j][2], v[j][3]), sc);
+            const uint32_t q0 = nearest_code<GENERAL>(cs, x0.x), q1 = nearest_code<GENERAL>(cs, x0.y);
+            const uint32_t q2 = nearest_code<GENERAL>(cs, x1.x), q3 = nearest_code<GENERAL>(cs, x1.y);
             if constexpr (K == 256) {
                 if (e + 4 <= n) {
-                    st_stream_u32(out + e, q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24));
+                    st_stream_u32(out + e, q0 | (q1 << 8) | (q2 << 16) | (q3 << 24));
                 } else {
-                    for (int i = 0; i < 4; i++)
-                        if (e + i < n) out[e + i] = (uint8_t)q[i];
+                    out[e] = (uint8_t)q0;
+                    if (e + 1 < n) out[e + 1] = (uint8_t)q1;
+                    if (e + 2 < n) out[e + 2] = (uint8_t)q2;
                 }
             } else {  // two 4-bit codes per byte, even element in the high nibble
-                uint8_t b0 = (uint8_t)((q[0] << 4) | (e + 1 < n ? q[1] : 0u));
-                uint8_t b1 = (uint8_t)((q[2] << 4) | (e + 3 < n ? q[3] : 0u));
+                const uint8_t b0 = (uint8_t)((q0 << 4) | (e + 1 < n ? q1 : 0u));
+                const uint8_t b1 = (uint8_t)((q2 << 4) | (e + 3 < n ? q3 : 0u));
                 uint8_t* o = out + (e >> 1);
                 if (e + 4 <= n) {
                     *reinterpret_cast<uint16_t*>(o) = (uint16_t)(b0 | (b1 << 8));
@@ -161,6 +158,22 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     }
 }
 
+template <int B, bool BF16, int K>
+__global__ void __launch_bounds__(kQThreads, 1)
+quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
+                float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CodeSmem& cs = *reinterpret_cast<CodeSmem*>(smem_raw);
+    float* red = reinterpret_cast<float*>(smem_raw + sizeof(CodeSmem));
+    bool fast, general;
+    if (!stage_one_code(cs, code, K, true, fast, general, flags)) return;
+    if (general)
+        quantize_loop<B, BF16, K, true>(cs, fast, A, n, absmax, out, red, flags);
+    else
+        quantize_loop<B, BF16, K, false>(cs, fast, A, n, absmax, out, red, flags);
+}
+
 // Dequantize: flat grid over 4-element chunks; each thread takes 4 chunks per pass.
 template <int K, bool BF16OUT>
 __global__ void __launch_bounds__(256)
@@ -169,8 +182,8 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
                   unsigned* flags)
 {
     __shared__ CodeSmem cs;
-    bool tiny;
-    if (!stage_one_code(cs, code, K, false, tiny, flags)) return;
+    bool fast, general;
+    if (!stage_one_code(cs, code, K, false, fast, general, flags)) return;
 
     const int64_t nchunks = (n + 3) / 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -243,13 +256,13 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
 }
 
 template <typename Kern>
-bnbq_status persistent_grid(Kern kern, int threads, int64_t work_units, int units_per_cta, int* grid)
+bnbq_status persistent_grid(Kern kern, int threads, size_t smem, int64_t work_units, int units_per_cta, int* grid)
 {
     int sms = 0;
     bnbq_status st = sm_count(&sms);
     if (st != BNBQ_OK) return st;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (per_sm < 1) per_sm = 1;
     int64_t need = (work_units + units_per_cta - 1) / units_per_cta;
@@ -266,11 +279,20 @@ bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax,
     unsigned* flags = nullptr;
     bnbq_status st = device_flag_ptr(&flags);
     if (st != BNBQ_OK) return st;
-    int grid = 0;
     auto kern = quantize_kernel<B, BF16, K>;
-    st = persistent_grid(kern, Geo::kThreads, (n + B - 1) / B, Geo::kGroups, &grid);
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    if (configured_dev != dev) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::kSmem);
+        if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(quantize smem)");
+        configured_dev = dev;
+    }
+    int grid = 0;
+    st = persistent_grid(kern, kQThreads, Geo::kSmem, (n + B - 1) / B, Geo::kGroups, &grid);
     if (st != BNBQ_OK) return st;
-    kern<<<grid, Geo::kThreads, 0, s>>>(code, A, n, absmax, out, flags);
+    kern<<<grid, kQThreads, Geo::kSmem, s>>>(code, A, n, absmax, out, flags);
     return cuda_status(cudaGetLastError(), "quantize_kernel launch");
 }
 
@@ -301,7 +323,7 @@ bnbq_status launch_dq(const float* code, const uint8_t* q, const float* absmax, 
     while ((1 << log2B) < B) log2B++;
     int grid = 0;
     auto kern = dequantize_kernel<K, BF16OUT>;
-    st = persistent_grid(kern, 256, (n + 3) / 4, 256 * 4, &grid);
+    st = persistent_grid(kern, 256, 0, (n + 3) / 4, 256 * 4, &grid);
     if (st != BNBQ_OK) return st;
     kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags);
     return cuda_status(cudaGetLastError(), "dequantize_kernel launch");

@@ -3,18 +3,23 @@
 // Method ("8-bit Optimizers via Block-wise Quantization", abstract, quoted on the blog.csdn.net
 // bitsandbytes guide, section 2): optimizer statistics are kept in 8 bits with block-wise
 // dynamic quantization while the update runs at 32-bit precision.  Per block this kernel
-//   loads p (fp32), g (fp32/bf16), the 8-bit codes and the two block scales,
-//   dequantizes m = code1[q1]*a1 and v = code2[q2]*a2 (codebooks staged in shared memory),
-//   applies the fp32 AdamW / Adam / Lion / momentum update and stores p at once,
-//   reduces the new block absmax of each state across the block's thread group,
-//   requantizes each state against its new absmax (nearest code) and stores codes and scales.
+//   loads p (fp32), g (fp32/bf16), the 8-bit codes and the block scales        (a4)
+//   dequantizes m = code1[q1]*a1 and v = code2[q2]*a2 from shared memory         (a4)
+//   applies the fp32 AdamW / Adam / Lion / momentum update and stores p at once   (a5)
+//   reduces the new block absmax of each state across the block's thread group     (a6)
+//   requantizes each state against its new absmax (nearest code) and stores it     (a7)
 // Tensors that keep 32-bit state (fewer than 4096 elements, and embedding tables: page
-// "Py之bitsandbytes…详细攻略", section "如果需要高精度的参数") are stepped by the same launch.
+// "Py之bitsandbytes…详细攻略", section "如果需要高精度的参数") are stepped by the same launch (a8).
 //
-// Scheduling: one launch per step for the whole tensor list.  The host uploads a table of
-// tensor descriptors (cached across steps); blocks are numbered globally, tensor by tensor, and
-// a persistent grid of SMs x resident CTAs strides over them.  Each block-group walks the
-// table with a monotone cursor, so finding a block's tensor costs nothing per element.
+// Layout and scheduling (a9): one launch per step for the whole tensor list.  The host uploads
+// a table of tensor descriptors (cached across steps); blocks are numbered globally, tensor by
+// tensor.  A persistent grid of kThreads-thread CTAs strides over them; a CTA holds
+// kThreads/(B/kEPT) block-groups of B/kEPT threads, each group owning one block at a time with
+// kEPT elements per thread (4-element chunks, consecutive across the group: every global access
+// is a fully coalesced vector access).  Groups synchronise with their own named barrier, so the
+// codebook tables are staged once per CTA and shared by all groups.  Each group walks the
+// descriptor table with a monotone cursor and keeps the current tensor's fields in registers.
+// Full blocks run without bounds checks; the last, partial block of a tensor takes a guarded path.
 //
 // Roofline: HBM.  AdamW with 8-bit state and bf16 gradients moves 14 bytes per element
 // (p read+write 8, g 2, q1 and q2 read+write 4) plus 16 bytes per block of scales.
@@ -23,297 +28,439 @@
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 
+#ifndef BNBQ_STEP_EPT
+#define BNBQ_STEP_EPT 16
+#endif
+#ifndef BNBQ_STEP_THREADS
+#define BNBQ_STEP_THREADS 512
+#endif
+#ifndef BNBQ_STEP_MIN_CTAS
+#define BNBQ_STEP_MIN_CTAS 1
+#endif
+
 namespace bnbq {
 namespace {
 
-constexpr int kEPT = 16;
+constexpr int kThreads = BNBQ_STEP_THREADS;
+constexpr int kEPT = BNBQ_STEP_EPT;   // elements per thread per block
+constexpr int kNCH = kEPT / 4;        // 4-element chunks per thread
+static_assert(kEPT % 4 == 0, "whole chunks");
 
 template <int B>
 struct SGeom {
-    static constexpr int G = B / kEPT;
-    static constexpr int kThreads = G < 128 ? 128 : G;
-    static constexpr int kGroups = kThreads / G;
-    static constexpr int kWarps = kThreads / 32;
+    static constexpr int G = B / kEPT;                 // threads per block-group
+    static constexpr int kGroups = kThreads / G;       // block-groups per CTA
+    static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
+    static_assert(kThreads % G == 0 && (G <= 32 || kGroups <= 15), "groups fit the CTA and the named barriers");
 };
 
 template <int OPT>
 struct OptTraits {
     static constexpr bool kTwoStates = (OPT == BNBQ_ADAMW || OPT == BNBQ_ADAM);
+    static constexpr int kCodes = kTwoStates ? 2 : 1;
 };
 
-// One element of the update.  Every binary32 operation is rounded on its own (explicit _rn
-// intrinsics, never contracted), in the order the header documents.
+// Scalars as pairs for the packed instructions.
+struct Pairs {
+    float2 b1, b2, omb1, omb2, decay, nstep, rcp_sqrt_bc2, nsqrt_bc2, eps, wd, nlr;
+};
+
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+
+__device__ __forceinline__ Pairs make_pairs(const StepScalars& sc)
+{
+    Pairs q;
+    q.b1 = f2(sc.b1); q.b2 = f2(sc.b2); q.omb1 = f2(sc.omb1); q.omb2 = f2(sc.omb2);
+    q.decay = f2(sc.decay); q.nstep = f2(-sc.step_size); q.rcp_sqrt_bc2 = f2(sc.rcp_sqrt_bc2);
+    q.nsqrt_bc2 = f2(-sc.sqrt_bc2); q.eps = f2(sc.eps); q.wd = f2(sc.wd); q.nlr = f2(-sc.lr);
+    return q;
+}
+
+// One pair of elements of the update.  Every binary32 operation is rounded on its own, in the
+// order the header documents; p - c*u is formed as p + (-c)*u, which rounds identically.
+// sqrt(v)/sqrt(1-b2^t) uses the FMA quotient: the host guarantees sqrt(1-b2^t) lies in
+// [2^-12, 1] (any binary32 b2 < 1), and sqrt(v) is 0 or at least 2^-75, so the quotient is exact.
 template <int OPT>
-__device__ __forceinline__ void update(const StepScalars& sc, float& p, float g, float& m, float& v)
+__device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, float2& p, float2 g,
+                                        float2& m, float2& v)
 {
     if constexpr (OPT == BNBQ_ADAMW || OPT == BNBQ_ADAM) {
         if constexpr (OPT == BNBQ_ADAM) {
-            if (sc.wd != 0.0f) g = __fadd_rn(g, __fmul_rn(sc.wd, p));
+            if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
         }
-        const float m1 = __fadd_rn(__fmul_rn(sc.b1, m), __fmul_rn(sc.omb1, g));
-        const float v1 = __fadd_rn(__fmul_rn(sc.b2, v), __fmul_rn(__fmul_rn(sc.omb2, g), g));
-        if constexpr (OPT == BNBQ_ADAMW) p = __fmul_rn(p, sc.decay);
-        const float s = __fsqrt_rn(v1);
-        const float sn = sc.bc2_fast ? div_markstein(s, sc.sqrt_bc2, sc.rcp_sqrt_bc2)
-                                     : __fdiv_rn(s, sc.sqrt_bc2);
-        const float den = __fadd_rn(sn, sc.eps);
-        p = __fsub_rn(p, __fmul_rn(sc.step_size, __fdiv_rn(m1, den)));
+        const float2 m1 = add2(mul2(k.b1, m), mul2(k.omb1, g));
+        const float2 v1 = add2(mul2(k.b2, v), mul2(mul2(k.omb2, g), g));
+        if constexpr (OPT == BNBQ_ADAMW) p = mul2(p, k.decay);
+        const float2 s = make_float2(__fsqrt_rn(v1.x), __fsqrt_rn(v1.y));
+        const float2 den = add2(div2_markstein(s, k.rcp_sqrt_bc2, k.nsqrt_bc2), k.eps);
+        const float2 u = make_float2(__fdiv_rn(m1.x, den.x), __fdiv_rn(m1.y, den.y));
+        p = add2(p, mul2(k.nstep, u));
         m = m1;
         v = v1;
     } else if constexpr (OPT == BNBQ_LION) {
-        const float c = __fadd_rn(__fmul_rn(sc.b1, m), __fmul_rn(sc.omb1, g));
-        const float sg = (c > 0.0f) ? 1.0f : ((c < 0.0f) ? -1.0f : 0.0f);
-        p = __fmul_rn(p, sc.decay);
-        p = __fsub_rn(p, __fmul_rn(sc.lr, sg));
-        m = __fadd_rn(__fmul_rn(sc.b2, m), __fmul_rn(sc.omb2, g));
+        const float2 c = add2(mul2(k.b1, m), mul2(k.omb1, g));
+        const float2 sg = make_float2((c.x > 0.0f) ? 1.0f : ((c.x < 0.0f) ? -1.0f : 0.0f),
+                                      (c.y > 0.0f) ? 1.0f : ((c.y < 0.0f) ? -1.0f : 0.0f));
+        p = mul2(p, k.decay);
+        p = add2(p, mul2(k.nlr, sg));
+        m = add2(mul2(k.b2, m), mul2(k.omb2, g));
     } else {  // momentum SGD, dampening 0
-        if (sc.wd != 0.0f) g = __fadd_rn(g, __fmul_rn(sc.wd, p));
-        const float m1 = __fadd_rn(__fmul_rn(sc.b1, m), g);
-        p = __fsub_rn(p, __fmul_rn(sc.lr, m1));
+        if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
+        const float2 m1 = add2(mul2(k.b1, m), g);
+        p = add2(p, mul2(k.nlr, m1));
         m = m1;
     }
 }
 
-__device__ __forceinline__ void load_p(const float* p, int64_t e, int64_t n, float (&v)[4])
+// ---- guarded element access for the partial last block of a tensor -----------------------------
+__device__ __forceinline__ float4 load_f4_guard(const float* p, int64_t e, int64_t n)
 {
-    if (e + 4 <= n) {
-        float4 f = ld_stream_f4(p + e);
-        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; i++) v[i] = (e + i < n) ? p[e + i] : 0.0f;
-    }
+    if (e + 4 <= n) return ld_stream_f4(p + e);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e + 0 < n) v.x = p[e + 0];
+    if (e + 1 < n) v.y = p[e + 1];
+    if (e + 2 < n) v.z = p[e + 2];
+    return v;
 }
 
-__device__ __forceinline__ void store_p(float* p, int64_t e, int64_t n, const float (&v)[4])
+__device__ __forceinline__ void store_f4_guard(float* p, int64_t e, int64_t n, float4 v)
 {
-    if (e + 4 <= n) {
-        st_stream_f4(p + e, make_float4(v[0], v[1], v[2], v[3]));
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-            if (e + i < n) p[e + i] = v[i];
-    }
+    if (e + 4 <= n) { st_stream_f4(p + e, v); return; }
+    if (e + 0 < n) p[e + 0] = v.x;
+    if (e + 1 < n) p[e + 1] = v.y;
+    if (e + 2 < n) p[e + 2] = v.z;
 }
 
-__device__ __forceinline__ void load_g(const void* g, bool bf16, int64_t e, int64_t n, float (&v)[4])
+__device__ __forceinline__ float4 load_g4(const void* g, bool bf16, int64_t e, int64_t n, bool full)
 {
-    if (e + 4 <= n) {
+    if (full || e + 4 <= n) {
         if (bf16) {
-            uint2 w = ld_stream_u2(static_cast<const uint16_t*>(g) + e);
-            v[0] = bf16lo_to_f32(w.x); v[1] = bf16hi_to_f32(w.x);
-            v[2] = bf16lo_to_f32(w.y); v[3] = bf16hi_to_f32(w.y);
-        } else {
-            float4 f = ld_stream_f4(static_cast<const float*>(g) + e);
-            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+            const uint2 w = ld_stream_u2(static_cast<const uint16_t*>(g) + e);
+            return make_float4(bf16lo_to_f32(w.x), bf16hi_to_f32(w.x), bf16lo_to_f32(w.y), bf16hi_to_f32(w.y));
         }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            float x = 0.0f;
-            if (e + i < n)
-                x = bf16 ? __uint_as_float((uint32_t)(static_cast<const uint16_t*>(g)[e + i]) << 16)
-                         : static_cast<const float*>(g)[e + i];
-            v[i] = x;
-        }
+        return ld_stream_f4(static_cast<const float*>(g) + e);
     }
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < 3; i++)
+        if (e + i < n)
+            v[i] = bf16 ? __uint_as_float((uint32_t)(static_cast<const uint16_t*>(g)[e + i]) << 16)
+                        : static_cast<const float*>(g)[e + i];
+    return make_float4(v[0], v[1], v[2], v[3]);
 }
 
-__device__ __forceinline__ uint32_t load_q(const uint8_t* q, int64_t e, int64_t n)
+__device__ __forceinline__ uint32_t load_q4(const uint8_t* q, int64_t e, int64_t n, bool full)
 {
-    if (e + 4 <= n) return ld_stream_u32(q + e);
+    if (full || e + 4 <= n) return ld_stream_u32(q + e);
     uint32_t w = 0;
-#pragma unroll
-    for (int i = 0; i < 4; i++)
+    for (int i = 0; i < 3; i++)
         if (e + i < n) w |= (uint32_t)q[e + i] << (8 * i);
     return w;
 }
 
-__device__ __forceinline__ void store_q(uint8_t* q, int64_t e, int64_t n, uint32_t w)
+__device__ __forceinline__ void store_q4(uint8_t* q, int64_t e, int64_t n, uint32_t w, bool full)
 {
-    if (e + 4 <= n) {
-        st_stream_u32(q + e, w);
+    if (full || e + 4 <= n) { st_stream_u32(q + e, w); return; }
+    for (int i = 0; i < 3; i++)
+        if (e + i < n) q[e + i] = (uint8_t)(w >> (8 * i));
+}
+
+__device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return __byte_perm(w, 0u, 0x4440u + (uint32_t)i); }
+
+// Group-wide max of (x, y) over the G threads of one block-group.
+template <int G, int NC>
+__device__ __forceinline__ void group_max2(float& x, float& y, int gi, int tg, int lane, unsigned gmask,
+                                           float* red, int& parity)
+{
+    if constexpr (G <= 32) {
+        x = group_max_nan<G>(x, gmask);
+        if constexpr (NC == 2) y = group_max_nan<G>(y, gmask);
     } else {
+        constexpr int W = G / 32;
+        x = group_max_nan<32>(x, 0xffffffffu);
+        if constexpr (NC == 2) y = group_max_nan<32>(y, 0xffffffffu);
+        float* r = red + ((gi * 2 + parity) * 2) * W;
+        const int w = tg >> 5;
+        if (lane == 0) {
+            r[w] = x;
+            if constexpr (NC == 2) r[W + w] = y;
+        }
+        group_barrier(1 + gi, G);
 #pragma unroll
-        for (int i = 0; i < 4; i++)
-            if (e + i < n) q[e + i] = (uint8_t)(w >> (8 * i));
+        for (int i = 0; i < W; i++) {
+            x = max_nan(x, r[i]);
+            if constexpr (NC == 2) y = max_nan(y, r[W + i]);
+        }
+        parity ^= 1;
+    }
+}
+
+// The current tensor's descriptor, held in registers while a group walks its blocks.
+struct Cur {
+    float* p;
+    const void* g;
+    uint8_t* q1;
+    uint8_t* q2;
+    float* a1;
+    float* a2;
+    int64_t n;
+    int first;
+    int next_first;  // first block of the next tensor (or INT_MAX)
+    int flags;
+};
+
+__device__ __forceinline__ void load_cur(Cur& c, const StepDesc* __restrict__ table, int i, int ntensors)
+{
+    const StepDesc* d = table + i;
+    c.p = d->p;
+    c.g = d->g;
+    c.q1 = static_cast<uint8_t*>(d->s1);
+    c.q2 = static_cast<uint8_t*>(d->s2);
+    c.a1 = d->a1;
+    c.a2 = d->a2;
+    c.n = d->n;
+    c.first = d->first_block;
+    c.flags = d->flags;
+    c.next_first = (i + 1 < ntensors) ? __ldg(&table[i + 1].first_block) : 0x7fffffff;
+}
+
+// Requantize the kNCH chunks of one block: FAST selects the FMA quotient.
+template <int OPT, int B, bool FULL, bool GENERAL, bool FAST>
+__device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, const CodeSmem& c1, const CodeSmem& c2,
+                                        const float2 (&mv)[2 * kNCH], const float2 (&vv)[2 * kNCH],
+                                        const BlockScale& s1, const BlockScale& s2)
+{
+    constexpr int G = SGeom<B>::G;
+    constexpr bool TWO = OptTraits<OPT>::kTwoStates;
+    const float2 r1 = f2(s1.r), na1 = f2(s1.na), r2 = f2(s2.r), na2 = f2(s2.na);
+#pragma unroll
+    for (int j = 0; j < kNCH; j++) {
+        const int64_t e = base + 4 * (j * G + tg);
+        if (!FULL && e >= c.n) continue;
+        uint32_t o1 = 0, o2 = 0;
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const float2 xn = FAST ? div2_markstein(mv[2 * j + h], r1, na1)
+                                   : make_float2(__fdiv_rn(mv[2 * j + h].x, s1.a), __fdiv_rn(mv[2 * j + h].y, s1.a));
+            o1 |= nearest_code<GENERAL>(c1, xn.x) << (16 * h);
+            o1 |= nearest_code<GENERAL>(c1, xn.y) << (16 * h + 8);
+            if constexpr (TWO) {
+                const float2 yn = FAST ? div2_markstein(vv[2 * j + h], r2, na2)
+                                       : make_float2(__fdiv_rn(vv[2 * j + h].x, s2.a), __fdiv_rn(vv[2 * j + h].y, s2.a));
+                o2 |= nearest_code<GENERAL>(c2, yn.x) << (16 * h);
+                o2 |= nearest_code<GENERAL>(c2, yn.y) << (16 * h + 8);
+            }
+        }
+        store_q4(c.q1, e, c.n, o1, FULL);
+        if constexpr (TWO) store_q4(c.q2, e, c.n, o2, FULL);
+    }
+}
+
+// One block with 8-bit state.  FULL: the block lies entirely inside the tensor.
+template <int OPT, int B, bool FULL, bool GENERAL>
+__device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp,
+                                       const CodeSmem* cs, bool fast1, bool fast2, int gi, int tg, int lane,
+                                       unsigned gmask, float* red, int& parity, unsigned* flags)
+{
+    constexpr int G = SGeom<B>::G;
+    constexpr bool TWO = OptTraits<OPT>::kTwoStates;
+    constexpr int NC = OptTraits<OPT>::kCodes;
+    const CodeSmem& c1 = cs[0];
+    const CodeSmem& c2 = cs[NC - 1];
+    const int64_t n = c.n;
+    const int64_t base = lb * B;
+    const bool gbf16 = (c.flags & kDescGBf16) != 0;
+
+    // a4: loads
+    float4 pv[kNCH], gv[kNCH];
+    uint32_t w1[kNCH], w2[kNCH];
+#pragma unroll
+    for (int j = 0; j < kNCH; j++) {
+        const int64_t e = base + 4 * (j * G + tg);
+        pv[j] = FULL ? ld_stream_f4(c.p + e) : load_f4_guard(c.p, e, n);
+        gv[j] = load_g4(c.g, gbf16, e, n, FULL);
+        w1[j] = load_q4(c.q1, e, n, FULL);
+        if constexpr (TWO) w2[j] = load_q4(c.q2, e, n, FULL);
+    }
+    const float a1 = __ldg(c.a1 + lb);
+    const float a2 = TWO ? __ldg(c.a2 + lb) : 0.0f;
+    const float2 a1p = f2(a1), a2p = f2(a2);
+
+    // a4 + a5: dequantize, update, store p
+    float2 mv[2 * kNCH], vv[2 * kNCH];
+    float mx1 = 0.0f, mx2 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kNCH; j++) {
+        const int64_t e = base + 4 * (j * G + tg);
+        float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
+        const float2 gh[2] = {make_float2(gv[j].x, gv[j].y), make_float2(gv[j].z, gv[j].w)};
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            float2 m = mul2(make_float2(c1.code[byte_of(w1[j], 2 * h)], c1.code[byte_of(w1[j], 2 * h + 1)]), a1p);
+            float2 v = make_float2(0.0f, 0.0f);
+            if constexpr (TWO)
+                v = mul2(make_float2(c2.code[byte_of(w2[j], 2 * h)], c2.code[byte_of(w2[j], 2 * h + 1)]), a2p);
+            update2<OPT>(sc, kp, ph[h], gh[h], m, v);
+            if (!FULL) {  // elements past the end do not count towards the block scale
+                if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }
+                if (e + 2 * h + 1 >= n) { m.y = 0.0f; v.y = 0.0f; }
+            }
+            mv[2 * j + h] = m;
+            vv[2 * j + h] = v;
+            mx1 = max_nan(mx1, max_nan(fabsf(m.x), fabsf(m.y)));
+            if constexpr (TWO) mx2 = max_nan(mx2, max_nan(fabsf(v.x), fabsf(v.y)));
+        }
+        const float4 po = make_float4(ph[0].x, ph[0].y, ph[1].x, ph[1].y);
+        if (FULL) {
+            st_stream_f4(c.p + e, po);
+        } else if (e < n) {
+            store_f4_guard(c.p, e, n, po);
+        }
+    }
+
+    // a6: block absmax of the new states
+    group_max2<G, NC>(mx1, mx2, gi, tg, lane, gmask, red, parity);
+    if (tg == 0) {
+        c.a1[lb] = mx1;
+        if constexpr (TWO) c.a2[lb] = mx2;
+        if (!(mx1 <= FLT_MAX) || !(mx2 <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
+    }
+
+    // a7: requantize (one block-uniform choice of quotient)
+    const BlockScale s1 = make_scale(mx1, fast1);
+    const BlockScale s2 = TWO ? make_scale(mx2, fast2) : s1;
+    if (s1.fast && s2.fast)
+        requant<OPT, B, FULL, GENERAL, true>(c, base, tg, c1, c2, mv, vv, s1, s2);
+    else
+        requant<OPT, B, FULL, GENERAL, false>(c, base, tg, c1, c2, mv, vv, s1, s2);
+}
+
+// One block with 32-bit state (no quantization).
+template <int OPT, int B>
+__device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp, int tg)
+{
+    constexpr int G = SGeom<B>::G;
+    constexpr bool TWO = OptTraits<OPT>::kTwoStates;
+    const int64_t n = c.n;
+    const int64_t base = lb * B;
+    float* m32 = reinterpret_cast<float*>(c.q1);
+    float* v32 = reinterpret_cast<float*>(c.q2);
+    const bool gbf16 = (c.flags & kDescGBf16) != 0;
+    const bool full = base + B <= n;
+#pragma unroll
+    for (int j = 0; j < kNCH; j++) {
+        const int64_t e = base + 4 * (j * G + tg);
+        if (e >= n) continue;
+        const float4 pv = load_f4_guard(c.p, e, n);
+        const float4 gv = load_g4(c.g, gbf16, e, n, full);
+        const float4 mq = load_f4_guard(m32, e, n);
+        const float4 vq = TWO ? load_f4_guard(v32, e, n) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 ph[2] = {make_float2(pv.x, pv.y), make_float2(pv.z, pv.w)};
+        float2 mh[2] = {make_float2(mq.x, mq.y), make_float2(mq.z, mq.w)};
+        float2 vh[2] = {make_float2(vq.x, vq.y), make_float2(vq.z, vq.w)};
+        update2<OPT>(sc, kp, ph[0], make_float2(gv.x, gv.y), mh[0], vh[0]);
+        update2<OPT>(sc, kp, ph[1], make_float2(gv.z, gv.w), mh[1], vh[1]);
+        store_f4_guard(c.p, e, n, make_float4(ph[0].x, ph[0].y, ph[1].x, ph[1].y));
+        store_f4_guard(m32, e, n, make_float4(mh[0].x, mh[0].y, mh[1].x, mh[1].y));
+        if constexpr (TWO) store_f4_guard(v32, e, n, make_float4(vh[0].x, vh[0].y, vh[1].x, vh[1].y));
+    }
+}
+
+template <int OPT, int B, bool GENERAL>
+__device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, int ntensors, int total_blocks,
+                                          const StepScalars& sc, const CodeSmem* cs, bool fast1, bool fast2,
+                                          float* red, unsigned* flags)
+{
+    using Geo = SGeom<B>;
+    constexpr int G = Geo::G;
+    const Pairs kp = make_pairs(sc);
+    const int gi = threadIdx.x / G;
+    const int tg = threadIdx.x % G;
+    const int lane = threadIdx.x & 31;
+    const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
+    int parity = 0;
+    int cur = 0;
+    Cur c;
+    load_cur(c, table, 0, ntensors);
+    for (int b = blockIdx.x * Geo::kGroups + gi; b < total_blocks; b += gridDim.x * Geo::kGroups) {
+        if (b >= c.next_first) {
+            do { cur++; } while (cur + 1 < ntensors && __ldg(&table[cur + 1].first_block) <= b);
+            load_cur(c, table, cur, ntensors);
+        }
+        const int64_t lb = (int64_t)(b - c.first);
+        if (c.flags & kDescState8) {
+            if ((lb + 1) * B <= c.n)
+                block8<OPT, B, true, GENERAL>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+            else
+                block8<OPT, B, false, GENERAL>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+        } else {
+            block32<OPT, B>(c, lb, sc, kp, tg);
+        }
     }
 }
 
 template <int OPT, int B>
-__global__ void __launch_bounds__(SGeom<B>::kThreads)
+__global__ void __launch_bounds__(kThreads, BNBQ_STEP_MIN_CTAS)
 step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, const StepScalars sc,
             const float* __restrict__ code1, const float* __restrict__ code2, unsigned* flags)
 {
-    using Geo = SGeom<B>;
-    constexpr int G = Geo::G;
-    constexpr bool TWO = OptTraits<OPT>::kTwoStates;
-    constexpr int NCODE = TWO ? 2 : 1;
-    __shared__ CodeSmem cs[NCODE];
-    __shared__ float red[2][NCODE][Geo::kWarps];
+    constexpr int NC = OptTraits<OPT>::kCodes;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CodeSmem* cs = reinterpret_cast<CodeSmem*>(smem_raw);
+    float* red = reinterpret_cast<float*>(cs + NC);
 
-    // a0: codebook stage (skipped when the list has no 8-bit tensor).
-    bool tiny[NCODE];
-    for (int c = 0; c < NCODE; c++) tiny[c] = false;
+    // a0: codebook stage (skipped when the list has no 8-bit tensor)
+    bool fast1 = true, fast2 = true, general = false;
     if (code1 != nullptr) {
         stage_code_pass1(cs[0], code1, 256);
-        if constexpr (TWO) stage_code_pass1(cs[1], code2, 256);
+        if constexpr (NC == 2) stage_code_pass1(cs[1], code2, 256);
         __syncthreads();
-        bool bad = false, t0 = false, t1 = false;
-        stage_code_pass2(cs[0], 256, bad, t0);
-        if constexpr (TWO) stage_code_pass2(cs[1], 256, bad, t1);
+        bool bad = false, t1 = false, t2 = false;
+        stage_code_pass2(cs[0], 256, bad, t1);
+        if constexpr (NC == 2) stage_code_pass2(cs[1], 256, bad, t2);
         bad = __syncthreads_or(bad);
-        tiny[0] = __syncthreads_or(t0);
-        if constexpr (TWO) tiny[NCODE - 1] = __syncthreads_or(t1);
+        fast1 = !__syncthreads_or(t1);
+        fast2 = !__syncthreads_or(t2);
         if (bad) {
             if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
             return;
         }
-        stage_code_pass3(cs[0], 256);
-        if constexpr (TWO) stage_code_pass3(cs[1], 256);
-        __syncthreads();
+        bool gen = stage_code_pass3(cs[0], 256);
+        if constexpr (NC == 2) gen |= stage_code_pass3(cs[1], 256);
+        general = __syncthreads_or(gen);
     }
-
-    const int gi = threadIdx.x / G;
-    const int tg = threadIdx.x % G;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
-    int parity = 0;
-    int cur = 0;
-
-    for (int b = blockIdx.x * Geo::kGroups + gi; b < total_blocks; b += gridDim.x * Geo::kGroups) {
-        while (cur + 1 < ntensors && __ldg(&table[cur + 1].first_block) <= b) cur++;
-        const StepDesc* d = table + cur;
-        float* p = d->p;
-        const void* gp = d->g;
-        const int64_t n = d->n;
-        const int dflags = d->flags;
-        const bool gbf16 = (dflags & kDescGBf16) != 0;
-        const int64_t lb = (int64_t)(b - d->first_block);
-        const int64_t base = lb * B;
-
-        if (dflags & kDescState8) {
-            // a4: load + dequantize
-            uint8_t* q1p = static_cast<uint8_t*>(d->s1);
-            uint8_t* q2p = static_cast<uint8_t*>(d->s2);
-            float pv[4][4], gv[4][4], mv[4][4], vv[4][4];
-            uint32_t w1[4], w2[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int64_t e = base + 4 * (j * G + tg);
-                load_p(p, e, n, pv[j]);
-                load_g(gp, gbf16, e, n, gv[j]);
-                w1[j] = load_q(q1p, e, n);
-                if constexpr (TWO) w2[j] = load_q(q2p, e, n);
-            }
-            const float a1 = __ldg(d->a1 + lb);
-            float a2 = 0.0f;
-            if constexpr (TWO) a2 = __ldg(d->a2 + lb);
-
-            // a5: update; p is stored at once
-            float mx1 = 0.0f, mx2 = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int64_t e = base + 4 * (j * G + tg);
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    float m = __fmul_rn(cs[0].code[(w1[j] >> (8 * i)) & 0xff], a1);
-                    float v = 0.0f;
-                    if constexpr (TWO) v = __fmul_rn(cs[NCODE - 1].code[(w2[j] >> (8 * i)) & 0xff], a2);
-                    update<OPT>(sc, pv[j][i], gv[j][i], m, v);
-                    if (e + i >= n) { m = 0.0f; v = 0.0f; }
-                    mv[j][i] = m;
-                    vv[j][i] = v;
-                    mx1 = max_nan(mx1, fabsf(m));
-                    if constexpr (TWO) mx2 = max_nan(mx2, fabsf(v));
-                }
-                if (e < n) store_p(p, e, n, pv[j]);
-            }
-
-            // a6: new block absmax of each state
-            if constexpr (G <= 32) {
-                mx1 = group_max_nan<G>(mx1, gmask);
-                if constexpr (TWO) mx2 = group_max_nan<G>(mx2, gmask);
-            } else {
-                mx1 = group_max_nan<32>(mx1, 0xffffffffu);
-                if constexpr (TWO) mx2 = group_max_nan<32>(mx2, 0xffffffffu);
-                if (lane == 0) {
-                    red[parity][0][warp] = mx1;
-                    if constexpr (TWO) red[parity][NCODE - 1][warp] = mx2;
-                }
-                __syncthreads();
-#pragma unroll
-                for (int w = 0; w < Geo::kWarps; w++) {
-                    mx1 = max_nan(mx1, red[parity][0][w]);
-                    if constexpr (TWO) mx2 = max_nan(mx2, red[parity][NCODE - 1][w]);
-                }
-                parity ^= 1;
-            }
-            if (tg == 0) {
-                d->a1[lb] = mx1;
-                if constexpr (TWO) d->a2[lb] = mx2;
-                if (!(mx1 <= FLT_MAX) || !(mx2 <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
-            }
-
-            // a7: requantize
-            const BlockScale s1 = make_scale(mx1, !tiny[0]);
-            BlockScale s2 = s1;
-            if constexpr (TWO) s2 = make_scale(mx2, !tiny[NCODE - 1]);
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int64_t e = base + 4 * (j * G + tg);
-                if (e >= n) continue;
-                uint32_t o1 = 0, o2 = 0;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    o1 |= nearest_code(cs[0], normalise(mv[j][i], s1)) << (8 * i);
-                    if constexpr (TWO) o2 |= nearest_code(cs[NCODE - 1], normalise(vv[j][i], s2)) << (8 * i);
-                }
-                store_q(q1p, e, n, o1);
-                if constexpr (TWO) store_q(q2p, e, n, o2);
-            }
-        } else {
-            // a8: 32-bit state path (same update, no quantization)
-            float* m32 = static_cast<float*>(d->s1);
-            float* v32 = static_cast<float*>(d->s2);
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int64_t e = base + 4 * (j * G + tg);
-                if (e >= n) continue;
-                float pv[4], gv[4], mv[4], vv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                load_p(p, e, n, pv);
-                load_g(gp, gbf16, e, n, gv);
-                load_p(m32, e, n, mv);
-                if constexpr (TWO) load_p(v32, e, n, vv);
-#pragma unroll
-                for (int i = 0; i < 4; i++) update<OPT>(sc, pv[i], gv[i], mv[i], vv[i]);
-                store_p(p, e, n, pv);
-                store_p(m32, e, n, mv);
-                if constexpr (TWO) store_p(v32, e, n, vv);
-            }
-        }
-    }
+    if (general)
+        step_loop<OPT, B, true>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+    else
+        step_loop<OPT, B, false>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
 }
 
 template <int OPT, int B>
-bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_blocks,
-                          const StepScalars& sc, const float* code1, const float* code2,
-                          cudaStream_t s)
+constexpr size_t step_smem_bytes()
+{
+    return OptTraits<OPT>::kCodes * sizeof(CodeSmem) +
+           sizeof(float) * SGeom<B>::kGroups * 2 * 2 * SGeom<B>::kGroupWarps;
+}
+
+template <int OPT, int B>
+bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_blocks, const StepScalars& sc,
+                          const float* code1, const float* code2, cudaStream_t s)
 {
     using Geo = SGeom<B>;
     unsigned* flags = nullptr;
     bnbq_status st = device_flag_ptr(&flags);
     if (st != BNBQ_OK) return st;
     auto kern = step_kernel<OPT, B>;
+    constexpr size_t smem = step_smem_bytes<OPT, B>();
     static thread_local int cached_dev = -1, cached_per_sm = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
     if (cached_dev != dev) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached_per_sm, kern, Geo::kThreads, 0);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(step smem)");
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached_per_sm, kern, kThreads, smem);
         if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-        if (cached_per_sm < 1) cached_per_sm = 1;
+        if (cached_per_sm < 1) return fail(BNBQ_ECUDA, "step kernel does not fit on an SM");
         cached_dev = dev;
     }
     int sms = 0;
@@ -322,7 +469,7 @@ bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_block
     const int64_t need = ((int64_t)total_blocks + Geo::kGroups - 1) / Geo::kGroups;
     const int64_t cap = (int64_t)sms * cached_per_sm;
     const int grid = (int)(need < cap ? need : cap);
-    kern<<<grid, Geo::kThreads, 0, s>>>(d_table, ntensors, total_blocks, sc, code1, code2, flags);
+    kern<<<grid, kThreads, smem, s>>>(d_table, ntensors, total_blocks, sc, code1, code2, flags);
     return cuda_status(cudaGetLastError(), "step_kernel launch");
 }
 
