@@ -86,18 +86,19 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def traffic_per_launch(workload: str, n_params: int):
+def traffic_per_launch(workload: str, algorithmic: int):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
-    kernel source (scaled from the captured case by parameters processed); else None."""
+    kernel source: the captured launch's DRAM bytes over its algorithmic bytes, times this
+    launch's algorithmic bytes (traffic grows in proportion to the parameters stepped)."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    e = d.get(workload.replace("_layer", "")) or d.get(workload)
+    e = d.get(workload)
     if not e or e.get("kernel_src_sha") != kernel_source_sha():
         return None
-    return int(round(e["dram_bytes_per_param"] * n_params))
+    return int(round(e["dram_over_algorithmic"] * algorithmic))
 
 
 # ------------------------------------------------------------------------------------ clocks
@@ -306,6 +307,7 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
     ev0.record(stream)
     for k in range(args.steps):
         t += 1
@@ -314,6 +316,7 @@ def main():
         k_end[k].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     barrier()
     clk = clocks.stop()
 
@@ -332,7 +335,7 @@ def main():
     peak, peak_kind = measured_peaks()
     achieved = alg / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload, lay.n_params),
+                "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload, alg),
                 "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes_per_launch": alg,
                 "kernel": f"step_kernel<{optim}, 2048>", "avg_launch_ms": round(avg_launch_ms, 4),
                 "min_launch_ms": round(min(launch_ms), 4), "max_launch_ms": round(max(launch_ms), 4)}

@@ -83,6 +83,49 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
     return true;
 }
 
+// Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division).
+template <int B, int K, bool GENERAL, bool FAST>
+__device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockScale& sc, const float (&v)[4][4],
+                                               int64_t base, int tg, int64_t n, uint8_t* __restrict__ out)
+{
+    constexpr int G = QGeom<B>::G;
+    const float2 r = make_float2(sc.r, sc.r), na = make_float2(sc.na, sc.na);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const int64_t e = base + 4 * (j * G + tg);
+        if (e >= n) continue;
+        float2 x0 = make_float2(v[j][0], v[j][1]), x1 = make_float2(v[j][2], v[j][3]);
+        if (FAST) {
+            x0 = div2_markstein(x0, r, na);
+            x1 = div2_markstein(x1, r, na);
+        } else {
+            x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
+            x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
+        }
+        const uint32_t q0 = nearest_code<GENERAL>(cs, x0.x), q1 = nearest_code<GENERAL>(cs, x0.y);
+        const uint32_t q2 = nearest_code<GENERAL>(cs, x1.x), q3 = nearest_code<GENERAL>(cs, x1.y);
+        if constexpr (K == 256) {
+            if (e + 4 <= n) {
+                st_stream_u32(out + e, q0 | (q1 << 8) | (q2 << 16) | (q3 << 24));
+            } else {
+                out[e] = (uint8_t)q0;
+                if (e + 1 < n) out[e + 1] = (uint8_t)q1;
+                if (e + 2 < n) out[e + 2] = (uint8_t)q2;
+            }
+        } else {  // two 4-bit codes per byte, even element in the high nibble
+            const uint8_t b0 = (uint8_t)((q0 << 4) | (e + 1 < n ? q1 : 0u));
+            const uint8_t b1 = (uint8_t)((q2 << 4) | (e + 3 < n ? q3 : 0u));
+            uint8_t* o = out + (e >> 1);
+            if (e + 4 <= n) {
+                *reinterpret_cast<uint16_t*>(o) = (uint16_t)(b0 | (b1 << 8));
+            } else {
+                o[0] = b0;
+                if (e + 2 < n) o[1] = b1;
+            }
+        }
+    }
+}
+
 template <int B, bool BF16, int K, bool GENERAL>
 __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
                                               float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
@@ -126,35 +169,10 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
             if (!(m <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
         }
         const BlockScale sc = make_scale(m, fast);
-
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int64_t e = base + 4 * (j * G + tg);
-            if (e >= n) continue;
-            const float2 x0 = normalise2(make_float2(v[j][0], v[j][1]), sc);
-            const float2 x1 = normalise2(make_float2(v[j][2], v[j][3]), sc);
-            const uint32_t q0 = nearest_code<GENERAL>(cs, x0.x), q1 = nearest_code<GENERAL>(cs, x0.y);
-            const uint32_t q2 = nearest_code<GENERAL>(cs, x1.x), q3 = nearest_code<GENERAL>(cs, x1.y);
-            if constexpr (K == 256) {
-                if (e + 4 <= n) {
-                    st_stream_u32(out + e, q0 | (q1 << 8) | (q2 << 16) | (q3 << 24));
-                } else {
-                    out[e] = (uint8_t)q0;
-                    if (e + 1 < n) out[e + 1] = (uint8_t)q1;
-                    if (e + 2 < n) out[e + 2] = (uint8_t)q2;
-                }
-            } else {  // two 4-bit codes per byte, even element in the high nibble
-                const uint8_t b0 = (uint8_t)((q0 << 4) | (e + 1 < n ? q1 : 0u));
-                const uint8_t b1 = (uint8_t)((q2 << 4) | (e + 3 < n ? q3 : 0u));
-                uint8_t* o = out + (e >> 1);
-                if (e + 4 <= n) {
-                    *reinterpret_cast<uint16_t*>(o) = (uint16_t)(b0 | (b1 << 8));
-                } else {
-                    o[0] = b0;
-                    if (e + 2 < n) o[1] = b1;
-                }
-            }
-        }
+        if (sc.fast)
+            quantize_store<B, K, GENERAL, true>(cs, sc, v, base, tg, n, out);
+        else
+            quantize_store<B, K, GENERAL, false>(cs, sc, v, base, tg, n, out);
     }
 }
 

@@ -32,7 +32,7 @@
 #define BNBQ_STEP_EPT 16
 #endif
 #ifndef BNBQ_STEP_THREADS
-#define BNBQ_STEP_THREADS 512
+#define BNBQ_STEP_THREADS 768
 #endif
 #ifndef BNBQ_STEP_MIN_CTAS
 #define BNBQ_STEP_MIN_CTAS 1
@@ -204,23 +204,24 @@ struct Cur {
     float* a2;
     int64_t n;
     int first;
-    int next_first;  // first block of the next tensor (or INT_MAX)
     int flags;
 };
 
 __device__ __forceinline__ void load_cur(Cur& c, const StepDesc* __restrict__ table, int i, int ntensors)
 {
     const StepDesc* d = table + i;
-    c.p = d->p;
-    c.g = d->g;
-    c.q1 = static_cast<uint8_t*>(d->s1);
-    c.q2 = static_cast<uint8_t*>(d->s2);
-    c.a1 = d->a1;
-    c.a2 = d->a2;
-    c.n = d->n;
-    c.first = d->first_block;
-    c.flags = d->flags;
-    c.next_first = (i + 1 < ntensors) ? __ldg(&table[i + 1].first_block) : 0x7fffffff;
+    auto ptr = [](const void* field) {
+        return reinterpret_cast<void*>(__ldg(reinterpret_cast<const unsigned long long*>(field)));
+    };
+    c.p = static_cast<float*>(ptr(&d->p));
+    c.g = ptr(&d->g);
+    c.q1 = static_cast<uint8_t*>(ptr(&d->s1));
+    c.q2 = static_cast<uint8_t*>(ptr(&d->s2));
+    c.a1 = static_cast<float*>(ptr(&d->a1));
+    c.a2 = static_cast<float*>(ptr(&d->a2));
+    c.n = __ldg(reinterpret_cast<const long long*>(&d->n));
+    c.first = __ldg(&d->first_block);
+    c.flags = __ldg(&d->flags);
 }
 
 // Requantize the kNCH chunks of one block: FAST selects the FMA quotient.
@@ -255,8 +256,46 @@ __device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, cons
     }
 }
 
-// One block with 8-bit state.  FULL: the block lies entirely inside the tensor.
-template <int OPT, int B, bool FULL, bool GENERAL>
+// Gradient chunk held in its loaded form until the update needs it.
+template <bool GB>
+struct GRaw;
+template <>
+struct GRaw<true> {
+    uint2 w;
+    __device__ __forceinline__ float2 half(int h) const
+    {
+        const uint32_t x = h ? w.y : w.x;
+        return make_float2(bf16lo_to_f32(x), bf16hi_to_f32(x));
+    }
+};
+template <>
+struct GRaw<false> {
+    float4 f;
+    __device__ __forceinline__ float2 half(int h) const { return h ? make_float2(f.z, f.w) : make_float2(f.x, f.y); }
+};
+
+template <bool GB, bool FULL>
+__device__ __forceinline__ GRaw<GB> load_graw(const void* g, int64_t e, int64_t n)
+{
+    GRaw<GB> r;
+    if constexpr (GB) {
+        const uint16_t* gh = static_cast<const uint16_t*>(g);
+        if (FULL || e + 4 <= n) {
+            r.w = ld_stream_u2(gh + e);
+        } else {
+            uint32_t v[3] = {0u, 0u, 0u};
+            for (int i = 0; i < 3; i++)
+                if (e + i < n) v[i] = gh[e + i];
+            r.w = make_uint2(v[0] | (v[1] << 16), v[2]);
+        }
+    } else {
+        r.f = FULL ? ld_stream_f4(static_cast<const float*>(g) + e) : load_f4_guard(static_cast<const float*>(g), e, n);
+    }
+    return r;
+}
+
+// One block with 8-bit state.  FULL: the block lies entirely inside the tensor; GB: bf16 grads.
+template <int OPT, int B, bool FULL, bool GENERAL, bool GB>
 __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp,
                                        const CodeSmem* cs, bool fast1, bool fast2, int gi, int tg, int lane,
                                        unsigned gmask, float* red, int& parity, unsigned* flags)
@@ -268,16 +307,17 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     const CodeSmem& c2 = cs[NC - 1];
     const int64_t n = c.n;
     const int64_t base = lb * B;
-    const bool gbf16 = (c.flags & kDescGBf16) != 0;
+    const int64_t e0 = base + 4 * tg;  // chunk j starts at e0 + 4*G*j
 
     // a4: loads
-    float4 pv[kNCH], gv[kNCH];
+    float4 pv[kNCH];
+    GRaw<GB> gv[kNCH];
     uint32_t w1[kNCH], w2[kNCH];
 #pragma unroll
     for (int j = 0; j < kNCH; j++) {
-        const int64_t e = base + 4 * (j * G + tg);
+        const int64_t e = e0 + 4 * G * j;
         pv[j] = FULL ? ld_stream_f4(c.p + e) : load_f4_guard(c.p, e, n);
-        gv[j] = load_g4(c.g, gbf16, e, n, FULL);
+        gv[j] = load_graw<GB, FULL>(c.g, e, n);
         w1[j] = load_q4(c.q1, e, n, FULL);
         if constexpr (TWO) w2[j] = load_q4(c.q2, e, n, FULL);
     }
@@ -290,16 +330,15 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     float mx1 = 0.0f, mx2 = 0.0f;
 #pragma unroll
     for (int j = 0; j < kNCH; j++) {
-        const int64_t e = base + 4 * (j * G + tg);
+        const int64_t e = e0 + 4 * G * j;
         float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
-        const float2 gh[2] = {make_float2(gv[j].x, gv[j].y), make_float2(gv[j].z, gv[j].w)};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             float2 m = mul2(make_float2(c1.code[byte_of(w1[j], 2 * h)], c1.code[byte_of(w1[j], 2 * h + 1)]), a1p);
             float2 v = make_float2(0.0f, 0.0f);
             if constexpr (TWO)
                 v = mul2(make_float2(c2.code[byte_of(w2[j], 2 * h)], c2.code[byte_of(w2[j], 2 * h + 1)]), a2p);
-            update2<OPT>(sc, kp, ph[h], gh[h], m, v);
+            update2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
             if (!FULL) {  // elements past the end do not count towards the block scale
                 if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }
                 if (e + 2 * h + 1 >= n) { m.y = 0.0f; v.y = 0.0f; }
@@ -379,19 +418,24 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
     const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
     int parity = 0;
     int cur = 0;
-    Cur c;
-    load_cur(c, table, 0, ntensors);
     for (int b = blockIdx.x * Geo::kGroups + gi; b < total_blocks; b += gridDim.x * Geo::kGroups) {
-        if (b >= c.next_first) {
-            do { cur++; } while (cur + 1 < ntensors && __ldg(&table[cur + 1].first_block) <= b);
-            load_cur(c, table, cur, ntensors);
-        }
+        while (cur + 1 < ntensors && __ldg(&table[cur + 1].first_block) <= b) cur++;
+        Cur c;
+        load_cur(c, table, cur, ntensors);
         const int64_t lb = (int64_t)(b - c.first);
         if (c.flags & kDescState8) {
-            if ((lb + 1) * B <= c.n)
-                block8<OPT, B, true, GENERAL>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
-            else
-                block8<OPT, B, false, GENERAL>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+            const bool full = (lb + 1) * B <= c.n;
+            if (c.flags & kDescGBf16) {
+                if (full)
+                    block8<OPT, B, true, GENERAL, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                else
+                    block8<OPT, B, false, GENERAL, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+            } else {
+                if (full)
+                    block8<OPT, B, true, GENERAL, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                else
+                    block8<OPT, B, false, GENERAL, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+            }
         } else {
             block32<OPT, B>(c, lb, sc, kp, tg);
         }
