@@ -25,7 +25,8 @@ CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DY
               "nf4": CODE_NF4, "linear": CODE_LINEAR}
 FLAG_BAD_CODE, FLAG_NONFINITE = 0x1, 0x2
 
-EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_codebook",
+EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_step_8bit_noalloc",
+            "bnbq_codebook",
             "bnbq_code_size", "bnbq_check_codebook", "bnbq_device_flags", "bnbq_last_error", "bnbq_release",
             "bnbq_version"]
 
@@ -76,6 +77,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.bnbq_dequantize_blockwise.argtypes = [vp, i32, vp, vp, i64, i32, vp, i32, vp]
         L.bnbq_step_8bit.argtypes = [i32, ctypes.POINTER(CTensor), i32, ctypes.POINTER(CHParams), i32, vp, vp,
                                      i32, vp]
+        L.bnbq_step_8bit_noalloc.argtypes = L.bnbq_step_8bit.argtypes
+        L.bnbq_step_8bit_noalloc.restype = i32
         for f in ("bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit",
                   "bnbq_check_codebook", "bnbq_device_flags"):
             getattr(L, f).restype = i32
@@ -218,6 +221,28 @@ def bnbq_step_8bit(opt: str | int, tensors: Sequence[TensorState] | ctypes.Array
     _check(lib().bnbq_step_8bit(o, arr, nt, ctypes.byref(hp), step,
                                 code1.data_ptr() if code1 is not None else None,
                                 code2.data_ptr() if code2 is not None else None, blocksize, _stream(stream)))
+
+
+def bnbq_step_8bit_noalloc(opt: str | int, tensors: Sequence[TensorState] | ctypes.Array, *, lr: float,
+                           beta1: float, beta2: float, eps: float, weight_decay: float, step: int,
+                           code1: Optional[torch.Tensor], code2: Optional[torch.Tensor], blocksize: int = 2048,
+                           stream=None, ntensors: Optional[int] = None) -> None:
+    """The same step as ``bnbq_step_8bit`` without any device allocation by the library (for
+    callers whose device memory all belongs to their own pool, or that must not allocate between
+    steps): the descriptor table lives in a fixed array inside the library (at most 4096
+    non-empty tensors per call).  All calls on a device share that array, so calls that can
+    overlap on the GPU must be ordered; the first call on a device does a one-time set-up and
+    should come before any stream capture."""
+    o = OPTIMS[opt] if isinstance(opt, str) else int(opt)
+    if isinstance(tensors, ctypes.Array):
+        arr, nt = tensors, ntensors
+    else:
+        arr, nt = pack_tensor_list(tensors), len(tensors)
+    hp = CHParams(lr, beta1, beta2, eps, weight_decay)
+    _check(lib().bnbq_step_8bit_noalloc(o, arr, nt, ctypes.byref(hp), step,
+                                        code1.data_ptr() if code1 is not None else None,
+                                        code2.data_ptr() if code2 is not None else None, blocksize,
+                                        _stream(stream)))
 
 
 def bnbq_device_flags(clear: bool = False) -> int:

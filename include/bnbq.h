@@ -147,6 +147,24 @@ BNBQ_API bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int
                            const bnbq_hparams* hp, int step, const float* code1,
                            const float* code2, int blocksize, bnbq_stream_t stream);
 
+/*
+ * bnbq_step_8bit_noalloc: the same step as bnbq_step_8bit (same arguments, same results) for
+ * callers that cannot let a library allocate device memory -- code whose device memory all
+ * belongs to its own pool or arena, processes that must not grow their footprint after start-up,
+ * or step loops that must never reach an allocator.  The pages describe no such entry point; it
+ * is this library's own.  Instead of an allocated, cached descriptor table it uses a fixed table
+ * compiled into the library: at most 4096 non-empty tensors per call (256 KiB of device memory
+ * on every GPU that loads the library, kept until the process exits); a longer list returns
+ * BNBQ_EINVAL.  It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on
+ * each device looks up the table's device address and sets the kernel's shared-memory limit; make
+ * that first call before capturing any stream.  All calls on a device share the one table and
+ * each call rewrites the entries it uses: calls whose work can overlap on the GPU (different
+ * streams with no ordering between them) race on it, so order them.
+ */
+BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnbq_tensor* list, int ntensors,
+                                            const bnbq_hparams* hp, int step, const float* code1,
+                                            const float* code2, int blocksize, bnbq_stream_t stream);
+
 /* Host-side codebook construction (out: host memory, 256 or 16 floats per bnbq_code_size).
  * Returns the number of values written, or -1 for an unknown kind / NULL out. */
 BNBQ_API int bnbq_codebook(bnbq_code_kind kind, float* out);
