@@ -102,8 +102,8 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
             x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
             x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
         }
-        const uint32_t q0 = nearest_code<GENERAL>(cs, x0.x), q1 = nearest_code<GENERAL>(cs, x0.y);
-        const uint32_t q2 = nearest_code<GENERAL>(cs, x1.x), q3 = nearest_code<GENERAL>(cs, x1.y);
+        const uint32_t q0 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x0.x), q1 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x0.y);
+        const uint32_t q2 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x1.x), q3 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x1.y);
         if constexpr (K == 256) {
             if (e + 4 <= n) {
                 st_stream_u32(out + e, q0 | (q1 << 8) | (q2 << 16) | (q3 << 24));

@@ -32,7 +32,10 @@
 #define BNBQ_STEP_EPT 16
 #endif
 #ifndef BNBQ_STEP_THREADS
-#define BNBQ_STEP_THREADS 768
+#define BNBQ_STEP_THREADS 768        // CTA size for blocksize 256 and 4096
+#endif
+#ifndef BNBQ_STEP_THREADS_2048
+#define BNBQ_STEP_THREADS_2048 BNBQ_STEP_THREADS  // CTA size for blocksize 2048
 #endif
 #ifndef BNBQ_STEP_MIN_CTAS
 #define BNBQ_STEP_MIN_CTAS 1
@@ -41,13 +44,13 @@
 namespace bnbq {
 namespace {
 
-constexpr int kThreads = BNBQ_STEP_THREADS;
 constexpr int kEPT = BNBQ_STEP_EPT;   // elements per thread per block
 constexpr int kNCH = kEPT / 4;        // 4-element chunks per thread
 static_assert(kEPT % 4 == 0, "whole chunks");
 
 template <int B>
 struct SGeom {
+    static constexpr int kThreads = (B == 2048) ? BNBQ_STEP_THREADS_2048 : BNBQ_STEP_THREADS;
     static constexpr int G = B / kEPT;                 // threads per block-group
     static constexpr int kGroups = kThreads / G;       // block-groups per CTA
     static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
@@ -224,8 +227,9 @@ __device__ __forceinline__ void load_cur(Cur& c, const StepDesc* __restrict__ ta
     c.flags = __ldg(&d->flags);
 }
 
-// Requantize the kNCH chunks of one block: FAST selects the FMA quotient.
-template <int OPT, int B, bool FULL, bool GENERAL, bool FAST>
+// Requantize the kNCH chunks of one block: FAST selects the FMA quotient; M1 / M2 are the
+// search modes of the two codebooks.
+template <int OPT, int B, bool FULL, int M1, int M2, bool FAST>
 __device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, const CodeSmem& c1, const CodeSmem& c2,
                                         const float2 (&mv)[2 * kNCH], const float2 (&vv)[2 * kNCH],
                                         const BlockScale& s1, const BlockScale& s2)
@@ -237,22 +241,22 @@ __device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, cons
     for (int j = 0; j < kNCH; j++) {
         const int64_t e = base + 4 * (j * G + tg);
         if (!FULL && e >= c.n) continue;
-        uint32_t o1 = 0, o2 = 0;
+        uint32_t w1[4], w2[4];
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const float2 xn = FAST ? div2_markstein(mv[2 * j + h], r1, na1)
                                    : make_float2(__fdiv_rn(mv[2 * j + h].x, s1.a), __fdiv_rn(mv[2 * j + h].y, s1.a));
-            o1 |= nearest_code<GENERAL>(c1, xn.x) << (16 * h);
-            o1 |= nearest_code<GENERAL>(c1, xn.y) << (16 * h + 8);
+            w1[2 * h] = nearest_code_word<M1>(c1, xn.x);
+            w1[2 * h + 1] = nearest_code_word<M1>(c1, xn.y);
             if constexpr (TWO) {
                 const float2 yn = FAST ? div2_markstein(vv[2 * j + h], r2, na2)
                                        : make_float2(__fdiv_rn(vv[2 * j + h].x, s2.a), __fdiv_rn(vv[2 * j + h].y, s2.a));
-                o2 |= nearest_code<GENERAL>(c2, yn.x) << (16 * h);
-                o2 |= nearest_code<GENERAL>(c2, yn.y) << (16 * h + 8);
+                w2[2 * h] = nearest_code_word<M2>(c2, yn.x);
+                w2[2 * h + 1] = nearest_code_word<M2>(c2, yn.y);
             }
         }
-        store_q4(c.q1, e, c.n, o1, FULL);
-        if constexpr (TWO) store_q4(c.q2, e, c.n, o2, FULL);
+        store_q4(c.q1, e, c.n, pack_top_bytes(w1[0], w1[1], w1[2], w1[3]), FULL);
+        if constexpr (TWO) store_q4(c.q2, e, c.n, pack_top_bytes(w2[0], w2[1], w2[2], w2[3]), FULL);
     }
 }
 
@@ -295,7 +299,7 @@ __device__ __forceinline__ GRaw<GB> load_graw(const void* g, int64_t e, int64_t 
 }
 
 // One block with 8-bit state.  FULL: the block lies entirely inside the tensor; GB: bf16 grads.
-template <int OPT, int B, bool FULL, bool GENERAL, bool GB>
+template <int OPT, int B, bool FULL, int M1, int M2, bool GB>
 __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp,
                                        const CodeSmem* cs, bool fast1, bool fast2, int gi, int tg, int lane,
                                        unsigned gmask, float* red, int& parity, unsigned* flags)
@@ -368,9 +372,9 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     const BlockScale s1 = make_scale(mx1, fast1);
     const BlockScale s2 = TWO ? make_scale(mx2, fast2) : s1;
     if (s1.fast && s2.fast)
-        requant<OPT, B, FULL, GENERAL, true>(c, base, tg, c1, c2, mv, vv, s1, s2);
+        requant<OPT, B, FULL, M1, M2, true>(c, base, tg, c1, c2, mv, vv, s1, s2);
     else
-        requant<OPT, B, FULL, GENERAL, false>(c, base, tg, c1, c2, mv, vv, s1, s2);
+        requant<OPT, B, FULL, M1, M2, false>(c, base, tg, c1, c2, mv, vv, s1, s2);
 }
 
 // One block with 32-bit state (no quantization).
@@ -404,7 +408,7 @@ __device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScal
     }
 }
 
-template <int OPT, int B, bool GENERAL>
+template <int OPT, int B, int M1, int M2>
 __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, int ntensors, int total_blocks,
                                           const StepScalars& sc, const CodeSmem* cs, bool fast1, bool fast2,
                                           float* red, unsigned* flags)
@@ -427,14 +431,14 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
             const bool full = (lb + 1) * B <= c.n;
             if (c.flags & kDescGBf16) {
                 if (full)
-                    block8<OPT, B, true, GENERAL, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                    block8<OPT, B, true, M1, M2, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
                 else
-                    block8<OPT, B, false, GENERAL, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                    block8<OPT, B, false, M1, M2, true>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
             } else {
                 if (full)
-                    block8<OPT, B, true, GENERAL, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                    block8<OPT, B, true, M1, M2, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
                 else
-                    block8<OPT, B, false, GENERAL, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
+                    block8<OPT, B, false, M1, M2, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
             }
         } else {
             block32<OPT, B>(c, lb, sc, kp, tg);
@@ -443,7 +447,7 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
 }
 
 template <int OPT, int B>
-__global__ void __launch_bounds__(kThreads, BNBQ_STEP_MIN_CTAS)
+__global__ void __launch_bounds__(SGeom<B>::kThreads, BNBQ_STEP_MIN_CTAS)
 step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, const StepScalars sc,
             const float* __restrict__ code1, const float* __restrict__ code2, unsigned* flags)
 {
@@ -453,7 +457,7 @@ step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, 
     float* red = reinterpret_cast<float*>(cs + NC);
 
     // a0: codebook stage (skipped when the list has no 8-bit tensor)
-    bool fast1 = true, fast2 = true, general = false;
+    bool fast1 = true, fast2 = true, general = false, nonneg2 = false;
     if (code1 != nullptr) {
         stage_code_pass1(cs[0], code1, 256);
         if constexpr (NC == 2) stage_code_pass1(cs[1], code2, 256);
@@ -471,11 +475,14 @@ step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, 
         bool gen = stage_code_pass3(cs[0], 256);
         if constexpr (NC == 2) gen |= stage_code_pass3(cs[1], 256);
         general = __syncthreads_or(gen);
+        nonneg2 = NC == 2 && cs[NC - 1].code[0] >= 0.0f;  // every code of the second state >= 0
     }
     if (general)
-        step_loop<OPT, B, true>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+        step_loop<OPT, B, kSearchGeneral, kSearchGeneral>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+    else if (nonneg2)
+        step_loop<OPT, B, kSearchSigned, kSearchNonNeg>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
     else
-        step_loop<OPT, B, false>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+        step_loop<OPT, B, kSearchSigned, kSearchSigned>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
 }
 
 template <int OPT, int B>
@@ -502,7 +509,7 @@ bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_block
     if (cached_dev != dev) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(step smem)");
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached_per_sm, kern, kThreads, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached_per_sm, kern, Geo::kThreads, smem);
         if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
         if (cached_per_sm < 1) return fail(BNBQ_ECUDA, "step kernel does not fit on an SM");
         cached_dev = dev;
@@ -513,7 +520,7 @@ bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_block
     const int64_t need = ((int64_t)total_blocks + Geo::kGroups - 1) / Geo::kGroups;
     const int64_t cap = (int64_t)sms * cached_per_sm;
     const int grid = (int)(need < cap ? need : cap);
-    kern<<<grid, kThreads, smem, s>>>(d_table, ntensors, total_blocks, sc, code1, code2, flags);
+    kern<<<grid, Geo::kThreads, smem, s>>>(d_table, ntensors, total_blocks, sc, code1, code2, flags);
     return cuda_status(cudaGetLastError(), "step_kernel launch");
 }
 
