@@ -49,6 +49,66 @@ WORKLOADS = {
     "llama7b_layer_adamw": ("llama7b_layer", "adamw", 4,
                             dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01), (0.0, 1.0)),
 }
+
+# Standalone quantize / dequantize sweep points (development measurements of those kernels):
+# name: (log2 n, input dtype, codebook, blocksize)
+QUANT_WORKLOADS = {
+    "quant_2p28_f32_signed_b2048": (28, "f32", "dynamic_signed", 2048),
+    "quant_2p28_bf16_signed_b2048": (28, "bf16", "dynamic_signed", 2048),
+    "quant_2p28_f32_nf4_b2048": (28, "f32", "nf4", 2048),
+    "quant_2p28_f32_signed_b256": (28, "f32", "dynamic_signed", 256),
+    "quant_2p28_f32_signed_b4096": (28, "f32", "dynamic_signed", 4096),
+}
+
+
+def bench_quant(args, base):
+    """Time bnbq_quantize_blockwise and bnbq_dequantize_blockwise on one sweep point (inputs far
+    above the L2 size for 2^28 elements); one JSON line with GB/s of each against the HBM peak."""
+    import torch
+    import block_wise_bit_b200 as bq
+    from block_wise_bit_b200 import workloads as W
+    log2n, dt, code_name, B = QUANT_WORKLOADS[args.workload]
+    n = 1 << log2n
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    dtype = torch.float32 if dt == "f32" else torch.bfloat16
+    x = W.normal(n, 1.0, dev, "quant-sweep", 1, args.workload)
+    W.outliers_(x, 0.001, 50.0, dev, "quant-sweep", 1, args.workload)
+    x = x.to(dtype)
+    code = bq.bnbq_codebook(code_name).to(dev)
+    K = code.numel()
+    absmax = torch.empty((n + B - 1) // B, dtype=torch.float32, device=dev)
+    q = torch.empty(n if K == 256 else (n + 1) // 2, dtype=torch.uint8, device=dev)
+    y = torch.empty(n, dtype=dtype, device=dev)
+    esz = x.element_size()
+    qbytes = n if K == 256 else n / 2
+    alg_q = n * esz + qbytes + 4 * absmax.numel()
+    alg_dq = qbytes + 4 * absmax.numel() + n * esz
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
+        bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        evs[k][0].record(stream)
+        bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
+        evs[k][1].record(stream)
+        bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
+        evs[k][2].record(stream)
+    torch.cuda.synchronize()
+    tq = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    td = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    peak, kind = measured_peaks()
+    out = dict(base, metric="block-wise quantize + dequantize elements/s", unit="elements/s",
+               value=n / ((tq + td) / 1e3), n_gpus=1, steps=args.steps, warmup=args.warmup,
+               ms_per_step=round(tq + td, 4), dtype=dt,
+               config={"workload": args.workload, "n": n, "blocksize": B, "codebook": code_name},
+               quantize={"ms": round(tq, 4), "GB/s": round(alg_q / tq / 1e6, 1), "frac": round(alg_q / tq / 1e6 / peak, 4)},
+               dequantize={"ms": round(td, 4), "GB/s": round(alg_dq / td / 1e6, 1), "frac": round(alg_dq / td / 1e6 / peak, 4)},
+               peak_gbs=peak, gpu_launches=2 * args.steps)
+    print(json.dumps(out))
+
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "block_wise_bit_b200", "csrc", f) for f in
                   ("bnbq_step.cu", "bnbq_device.cuh", "bnbq_internal.h")]
@@ -215,7 +275,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama7b_adamw")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS), default="llama7b_adamw")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -227,7 +287,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS[args.workload]
+    if args.workload in QUANT_WORKLOADS:
+        shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS["llama7b_adamw"]
+    else:
+        shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS[args.workload]
 
     from block_wise_bit_b200 import workloads as W
     lay = W.Layout.build(W.SHAPES[shape](), 2048)
@@ -266,6 +329,9 @@ def main():
     import torch.distributed as dist
     import block_wise_bit_b200 as bq
     from block_wise_bit_b200.optim import FlatStateList
+
+    if args.workload.startswith("quant"):
+        return bench_quant(args, base)
 
     if world > 1:
         from datetime import timedelta

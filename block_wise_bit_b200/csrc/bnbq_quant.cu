@@ -84,7 +84,7 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
 }
 
 // Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division).
-template <int B, int K, bool GENERAL, bool FAST>
+template <int B, int K, int MODE, bool FAST>
 __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockScale& sc, const float (&v)[4][4],
                                                int64_t base, int tg, int64_t n, uint8_t* __restrict__ out)
 {
@@ -102,17 +102,19 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
             x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
             x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
         }
-        const uint32_t q0 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x0.x), q1 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x0.y);
-        const uint32_t q2 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x1.x), q3 = nearest_code<GENERAL ? kSearchGeneral : kSearchSigned>(cs, x1.y);
+        const uint32_t w0 = nearest_code_word<MODE>(cs, x0.x), w1 = nearest_code_word<MODE>(cs, x0.y);
+        const uint32_t w2 = nearest_code_word<MODE>(cs, x1.x), w3 = nearest_code_word<MODE>(cs, x1.y);
         if constexpr (K == 256) {
+            const uint32_t word = pack_top_bytes(w0, w1, w2, w3);
             if (e + 4 <= n) {
-                st_stream_u32(out + e, q0 | (q1 << 8) | (q2 << 16) | (q3 << 24));
+                st_stream_u32(out + e, word);
             } else {
-                out[e] = (uint8_t)q0;
-                if (e + 1 < n) out[e + 1] = (uint8_t)q1;
-                if (e + 2 < n) out[e + 2] = (uint8_t)q2;
+                out[e] = (uint8_t)word;
+                if (e + 1 < n) out[e + 1] = (uint8_t)(word >> 8);
+                if (e + 2 < n) out[e + 2] = (uint8_t)(word >> 16);
             }
         } else {  // two 4-bit codes per byte, even element in the high nibble
+            const uint32_t q0 = w0 >> 24, q1 = w1 >> 24, q2 = w2 >> 24, q3 = w3 >> 24;
             const uint8_t b0 = (uint8_t)((q0 << 4) | (e + 1 < n ? q1 : 0u));
             const uint8_t b1 = (uint8_t)((q2 << 4) | (e + 3 < n ? q3 : 0u));
             uint8_t* o = out + (e >> 1);
@@ -126,7 +128,7 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
     }
 }
 
-template <int B, bool BF16, int K, bool GENERAL>
+template <int B, bool BF16, int K, int MODE>
 __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
                                               float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
                                               unsigned* flags)
@@ -170,9 +172,9 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
         }
         const BlockScale sc = make_scale(m, fast);
         if (sc.fast)
-            quantize_store<B, K, GENERAL, true>(cs, sc, v, base, tg, n, out);
+            quantize_store<B, K, MODE, true>(cs, sc, v, base, tg, n, out);
         else
-            quantize_store<B, K, GENERAL, false>(cs, sc, v, base, tg, n, out);
+            quantize_store<B, K, MODE, false>(cs, sc, v, base, tg, n, out);
     }
 }
 
@@ -187,9 +189,11 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     bool fast, general;
     if (!stage_one_code(cs, code, K, true, fast, general, flags)) return;
     if (general)
-        quantize_loop<B, BF16, K, true>(cs, fast, A, n, absmax, out, red, flags);
+        quantize_loop<B, BF16, K, kSearchGeneral>(cs, fast, A, n, absmax, out, red, flags);
+    else if (cs.code[0] >= 0.0f)  // every code >= 0
+        quantize_loop<B, BF16, K, kSearchNonNeg>(cs, fast, A, n, absmax, out, red, flags);
     else
-        quantize_loop<B, BF16, K, false>(cs, fast, A, n, absmax, out, red, flags);
+        quantize_loop<B, BF16, K, kSearchSigned>(cs, fast, A, n, absmax, out, red, flags);
 }
 
 // Dequantize: flat grid over 4-element chunks; each thread takes 4 chunks per pass.
