@@ -179,7 +179,7 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
 }
 
 template <int B, bool BF16, int K>
-__global__ void __launch_bounds__(kQThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 2)
 quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
                 float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags)
 {
