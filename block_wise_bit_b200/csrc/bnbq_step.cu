@@ -115,6 +115,38 @@ __device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, f
     }
 }
 
+// ---- codebook tables of the step kernel ---------------------------------------------------------
+// The bucket tables hold only the indices that a normalised value in [-1, 1] reaches: the signed
+// table of the first state [kSignedLo, kSignedHi] and, for a second codebook without negative
+// codes, the non-negative table [kNonNegLo, kSignedHi] (about 44 KB for both).  The padding
+// around them keeps every index that any bit pattern can form ([-kHalf, kHalf) around each
+// table's index 0) inside the allocation.  A small footprint matters here: the CTA's share of
+// the SM's unified L1/shared memory left to L1 is where the streamed loads land while in flight.
+template <int NC>
+struct StepSmem {
+    float code[NC][256];
+    float mid[NC][256];
+    uint32_t pad0[NC == 2 ? 4 : 260];
+    uint32_t stab[kSignedHi - kSignedLo + 1];
+    uint32_t utab[NC == 2 ? kSignedHi - kNonNegLo + 1 : 4];
+    uint32_t pad1[128];
+
+    __device__ __forceinline__ const uint32_t* center1() const { return stab - kSignedLo; }
+    __device__ __forceinline__ const uint32_t* center2() const { return utab - kNonNegLo; }
+};
+
+// The second state's codebook has negative codes: binary search over its midpoints.
+constexpr int kSearchBinary = 3;
+
+template <int MODE>
+__device__ __forceinline__ uint32_t step_code_word(const uint32_t* center, const float* mid, float x)
+{
+    if constexpr (MODE == kSearchBinary)
+        return (uint32_t)count_mid_below(mid, 256, x) << 24;
+    else
+        return nearest_code_word<MODE>(center, mid, x);
+}
+
 // ---- guarded element access for the partial last block of a tensor -----------------------------
 __device__ __forceinline__ float4 load_f4_guard(const float* p, int64_t e, int64_t n)
 {
@@ -230,13 +262,17 @@ __device__ __forceinline__ void load_cur(Cur& c, const StepDesc* __restrict__ ta
 // Requantize the kNCH chunks of one block: FAST selects the FMA quotient; M1 / M2 are the
 // search modes of the two codebooks.
 template <int OPT, int B, bool FULL, int M1, int M2, bool FAST>
-__device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, const CodeSmem& c1, const CodeSmem& c2,
+__device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, const StepSmem<OptTraits<OPT>::kCodes>& sm,
                                         const float2 (&mv)[2 * kNCH], const float2 (&vv)[2 * kNCH],
                                         const BlockScale& s1, const BlockScale& s2)
 {
     constexpr int G = SGeom<B>::G;
     constexpr bool TWO = OptTraits<OPT>::kTwoStates;
     const float2 r1 = f2(s1.r), na1 = f2(s1.na), r2 = f2(s2.r), na2 = f2(s2.na);
+    const uint32_t* t1 = sm.center1();
+    const uint32_t* t2 = sm.center2();
+    const float* mid1 = sm.mid[0];
+    const float* mid2 = sm.mid[TWO ? 1 : 0];
 #pragma unroll
     for (int j = 0; j < kNCH; j++) {
         const int64_t e = base + 4 * (j * G + tg);
@@ -246,13 +282,13 @@ __device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, cons
         for (int h = 0; h < 2; h++) {
             const float2 xn = FAST ? div2_markstein(mv[2 * j + h], r1, na1)
                                    : make_float2(__fdiv_rn(mv[2 * j + h].x, s1.a), __fdiv_rn(mv[2 * j + h].y, s1.a));
-            w1[2 * h] = nearest_code_word<M1>(c1, xn.x);
-            w1[2 * h + 1] = nearest_code_word<M1>(c1, xn.y);
+            w1[2 * h] = step_code_word<M1>(t1, mid1, xn.x);
+            w1[2 * h + 1] = step_code_word<M1>(t1, mid1, xn.y);
             if constexpr (TWO) {
                 const float2 yn = FAST ? div2_markstein(vv[2 * j + h], r2, na2)
                                        : make_float2(__fdiv_rn(vv[2 * j + h].x, s2.a), __fdiv_rn(vv[2 * j + h].y, s2.a));
-                w2[2 * h] = nearest_code_word<M2>(c2, yn.x);
-                w2[2 * h + 1] = nearest_code_word<M2>(c2, yn.y);
+                w2[2 * h] = step_code_word<M2>(t2, mid2, yn.x);
+                w2[2 * h + 1] = step_code_word<M2>(t2, mid2, yn.y);
             }
         }
         store_q4(c.q1, e, c.n, pack_top_bytes(w1[0], w1[1], w1[2], w1[3]), FULL);
@@ -301,14 +337,14 @@ __device__ __forceinline__ GRaw<GB> load_graw(const void* g, int64_t e, int64_t 
 // One block with 8-bit state.  FULL: the block lies entirely inside the tensor; GB: bf16 grads.
 template <int OPT, int B, bool FULL, int M1, int M2, bool GB>
 __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp,
-                                       const CodeSmem* cs, bool fast1, bool fast2, int gi, int tg, int lane,
-                                       unsigned gmask, float* red, int& parity, unsigned* flags)
+                                       const StepSmem<OptTraits<OPT>::kCodes>& cs, bool fast1, bool fast2, int gi,
+                                       int tg, int lane, unsigned gmask, float* red, int& parity, unsigned* flags)
 {
     constexpr int G = SGeom<B>::G;
     constexpr bool TWO = OptTraits<OPT>::kTwoStates;
     constexpr int NC = OptTraits<OPT>::kCodes;
-    const CodeSmem& c1 = cs[0];
-    const CodeSmem& c2 = cs[NC - 1];
+    const float* code1 = cs.code[0];
+    const float* code2 = cs.code[NC - 1];
     const int64_t n = c.n;
     const int64_t base = lb * B;
     const int64_t e0 = base + 4 * tg;  // chunk j starts at e0 + 4*G*j
@@ -338,10 +374,10 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
         float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            float2 m = mul2(make_float2(c1.code[byte_of(w1[j], 2 * h)], c1.code[byte_of(w1[j], 2 * h + 1)]), a1p);
+            float2 m = mul2(make_float2(code1[byte_of(w1[j], 2 * h)], code1[byte_of(w1[j], 2 * h + 1)]), a1p);
             float2 v = make_float2(0.0f, 0.0f);
             if constexpr (TWO)
-                v = mul2(make_float2(c2.code[byte_of(w2[j], 2 * h)], c2.code[byte_of(w2[j], 2 * h + 1)]), a2p);
+                v = mul2(make_float2(code2[byte_of(w2[j], 2 * h)], code2[byte_of(w2[j], 2 * h + 1)]), a2p);
             update2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
             if (!FULL) {  // elements past the end do not count towards the block scale
                 if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }
@@ -372,9 +408,9 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     const BlockScale s1 = make_scale(mx1, fast1);
     const BlockScale s2 = TWO ? make_scale(mx2, fast2) : s1;
     if (s1.fast && s2.fast)
-        requant<OPT, B, FULL, M1, M2, true>(c, base, tg, c1, c2, mv, vv, s1, s2);
+        requant<OPT, B, FULL, M1, M2, true>(c, base, tg, cs, mv, vv, s1, s2);
     else
-        requant<OPT, B, FULL, M1, M2, false>(c, base, tg, c1, c2, mv, vv, s1, s2);
+        requant<OPT, B, FULL, M1, M2, false>(c, base, tg, cs, mv, vv, s1, s2);
 }
 
 // One block with 32-bit state (no quantization).
@@ -410,8 +446,8 @@ __device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScal
 
 template <int OPT, int B, int M1, int M2>
 __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, int ntensors, int total_blocks,
-                                          const StepScalars& sc, const CodeSmem* cs, bool fast1, bool fast2,
-                                          float* red, unsigned* flags)
+                                          const StepScalars& sc, const StepSmem<OptTraits<OPT>::kCodes>& cs,
+                                          bool fast1, bool fast2, float* red, unsigned* flags)
 {
     using Geo = SGeom<B>;
     constexpr int G = Geo::G;
@@ -453,18 +489,18 @@ step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, 
 {
     constexpr int NC = OptTraits<OPT>::kCodes;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    CodeSmem* cs = reinterpret_cast<CodeSmem*>(smem_raw);
-    float* red = reinterpret_cast<float*>(cs + NC);
+    StepSmem<NC>& cs = *reinterpret_cast<StepSmem<NC>*>(smem_raw);
+    float* red = reinterpret_cast<float*>(smem_raw + sizeof(StepSmem<NC>));
 
     // a0: codebook stage (skipped when the list has no 8-bit tensor)
-    bool fast1 = true, fast2 = true, general = false, nonneg2 = false;
+    bool fast1 = true, fast2 = true, general = false, nonneg2 = true;
     if (code1 != nullptr) {
-        stage_code_pass1(cs[0], code1, 256);
-        if constexpr (NC == 2) stage_code_pass1(cs[1], code2, 256);
+        stage_codes(cs.code[0], code1, 256);
+        if constexpr (NC == 2) stage_codes(cs.code[1], code2, 256);
         __syncthreads();
         bool bad = false, t1 = false, t2 = false;
-        stage_code_pass2(cs[0], 256, bad, t1);
-        if constexpr (NC == 2) stage_code_pass2(cs[1], 256, bad, t2);
+        stage_midpoints(cs.code[0], cs.mid[0], 256, bad, t1);
+        if constexpr (NC == 2) stage_midpoints(cs.code[1], cs.mid[1], 256, bad, t2);
         bad = __syncthreads_or(bad);
         fast1 = !__syncthreads_or(t1);
         fast2 = !__syncthreads_or(t2);
@@ -472,23 +508,23 @@ step_kernel(const StepDesc* __restrict__ table, int ntensors, int total_blocks, 
             if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
             return;
         }
-        bool gen = stage_code_pass3(cs[0], 256);
-        if constexpr (NC == 2) gen |= stage_code_pass3(cs[1], 256);
+        nonneg2 = NC == 1 || cs.code[NC - 1][0] >= 0.0f;  // every code of the second state >= 0
+        bool gen = build_bucket_entries(cs.stab - kSignedLo, cs.mid[0], 256, kSignedLo, kSignedHi);
+        if (NC == 2 && nonneg2) gen |= build_bucket_entries(cs.utab - kNonNegLo, cs.mid[NC - 1], 256, kNonNegLo, kSignedHi);
         general = __syncthreads_or(gen);
-        nonneg2 = NC == 2 && cs[NC - 1].code[0] >= 0.0f;  // every code of the second state >= 0
     }
-    if (general)
+    if (!nonneg2)
+        step_loop<OPT, B, kSearchGeneral, kSearchBinary>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+    else if (general)
         step_loop<OPT, B, kSearchGeneral, kSearchGeneral>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
-    else if (nonneg2)
-        step_loop<OPT, B, kSearchSigned, kSearchNonNeg>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
     else
-        step_loop<OPT, B, kSearchSigned, kSearchSigned>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
+        step_loop<OPT, B, kSearchSigned, kSearchNonNeg>(table, ntensors, total_blocks, sc, cs, fast1, fast2, red, flags);
 }
 
 template <int OPT, int B>
 constexpr size_t step_smem_bytes()
 {
-    return OptTraits<OPT>::kCodes * sizeof(CodeSmem) +
+    return sizeof(StepSmem<OptTraits<OPT>::kCodes>) +
            sizeof(float) * SGeom<B>::kGroups * 2 * 2 * SGeom<B>::kGroupWarps;
 }
 

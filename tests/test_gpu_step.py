@@ -128,11 +128,11 @@ def test_tiny_adamw_trajectory_and_quantize():
 SIZES = [1, 3, 5, 4095, 4096, 4100, 2048 * 3 + 17, 65536, 70001]
 
 
-def _small_list(optim, B, g_dtype, seed):
+def _small_list(optim, B, g_dtype, seed, codes=None):
     """Tensors of SIZES (policy: < 4096 -> 32-bit) plus one large tensor forced to 32-bit, with
     a synthetic non-zero state."""
     two = optim in ("adamw", "adam")
-    c1, c2 = _codes()
+    c1, c2 = codes if codes is not None else _codes()
     out = []
     for i, n in enumerate(SIZES + [30000]):
         bits = 32 if (n < 4096 or i == len(SIZES)) else 8
@@ -143,6 +143,8 @@ def _small_list(optim, B, g_dtype, seed):
             s1 = W.random_codes(n, DEV, "small", seed, i, "q1")
             a1 = W.log_uniform(nb, 1e-4, 1e-2, DEV, "small", seed, i, "a1")
             s2 = W.random_codes(n, DEV, "small", seed, i, "q2") if two else None
+            if two and float(c2[0]) < 0:  # a signed second codebook: start v >= 0 (codes 128..255)
+                s2 = s2 % 128 + 128
             a2 = W.log_uniform(nb, 1e-8, 1e-5, DEV, "small", seed, i, "a2") if two else None
             if optim == "momentum":
                 a1 = W.log_uniform(nb, 1e-3, 1e-1, DEV, "small", seed, i, "a1m")
@@ -172,6 +174,57 @@ def test_small_list_all_optimizers(optim, B, g_dtype):
             parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(),
                                      c2.numpy() if two else None, B, HP[optim], t)
             _compare(f"{optim}/B{B}/{g_dtype}/#{i}(n={ts.p.numel()})", ts, ht, g_np, optim, B, t, c1.numpy(),
+                     c2.numpy() if two else None, prev)
+
+
+def _clustered(signed):
+    """A linear codebook (signed: -1 + 2k/255; unsigned: k/255) with two codes moved so that two
+    decision midpoints fall inside one bucket of the table (the binary32 values sharing the
+    16-bit prefix of [0.498046875, 0.5)): the step must take its general search."""
+    if signed:
+        c = np.array([-1 + 2 * k / 255 for k in range(256)])
+        c[192], c[193] = 0.499, 0.5
+    else:
+        c = np.array([k / 255 for k in range(256)])
+        c[128], c[129] = 0.499, 0.5
+    c = c.astype(np.float32)
+    assert np.all(np.diff(c) > 0)
+    return torch.from_numpy(c)
+
+
+CODE_MODES = {
+    # second codebook with negative codes: binary search for the second state
+    "signed-signed": lambda: (bq.bnbq_codebook("dynamic_signed"), bq.bnbq_codebook("dynamic_signed")),
+    # a midpoint in the merged bucket of tiny magnitudes (linear codes around 0): general search
+    "linear-linear": lambda: (bq.bnbq_codebook("linear"), bq.bnbq_codebook("linear")),
+    # two midpoints in one bucket of the first / the second codebook: general search
+    "clustered-unsigned": lambda: (_clustered(True), bq.bnbq_codebook("dynamic_unsigned")),
+    "signed-clustered": lambda: (bq.bnbq_codebook("dynamic_signed"), _clustered(False)),
+}
+
+
+@pytest.mark.parametrize("mode", sorted(CODE_MODES))
+@pytest.mark.parametrize("optim", ["adamw", "lion"])
+def test_small_list_other_codebooks(mode, optim):
+    """Codebooks that the bucket tables cannot serve with their single-compare rule take the
+    general (walk) or binary search; results must still match the oracle."""
+    B = 2048
+    c1, c2 = CODE_MODES[mode]()
+    if optim == "lion" and mode in ("signed-signed", "signed-clustered"):
+        pytest.skip("one state: the second codebook is unused")
+    tensors, c1, c2 = _small_list(optim, B, torch.bfloat16, 11, codes=(c1, c2))
+    hts = [HostTensor(ts) for ts in tensors]
+    two = optim in ("adamw", "adam")
+    for t in (1, 2):
+        prevs = [_copy_prev(h) for h in hts]
+        bq.bnbq_step_8bit(optim, tensors, step=t, code1=c1.to(DEV), code2=c2.to(DEV) if two else None, blocksize=B,
+                          **HP[optim])
+        torch.cuda.synchronize()
+        for i, (ts, ht, prev) in enumerate(zip(tensors, hts, prevs)):
+            g_np = parity.to_np(ts.g)
+            parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(),
+                                     c2.numpy() if two else None, B, HP[optim], t)
+            _compare(f"{optim}/{mode}/#{i}(n={ts.p.numel()})", ts, ht, g_np, optim, B, t, c1.numpy(),
                      c2.numpy() if two else None, prev)
 
 
