@@ -22,9 +22,9 @@ _SRC = os.path.join(_HERE, "bnbq_oracle.c")
 _HDR = os.path.join(_HERE, "bnbq_oracle.h")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-ADAMW, ADAM, LION, MOMENTUM = 0, 1, 2, 3
+ADAMW, ADAM, LION, MOMENTUM, RMSPROP = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
-OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM}
+OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM, "rmsprop": RMSPROP}
 
 _lock = threading.Lock()
 _lib = None

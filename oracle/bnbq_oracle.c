@@ -255,6 +255,9 @@ int oracle_dequantize_blockwise(const float* code, int K, const uint8_t* q, cons
  *        m' = b2*m + (1-b2)*g.
  *   Momentum SGD (the "exponentially smoothed sum" of [BWQ]; dampening 0): g = g + wd*p if
  *        wd != 0 ; m' = b1*m + g ; p = p - lr*m'.
+ *   RMSprop [RMSP] (one state, the running mean of squares, kept with the unsigned code; b1
+ *        carries the smoothing constant alpha): g = g + wd*p if wd != 0 ;
+ *        v' = b1*v + ((1-b1)*g)*g ; p = p - lr * (g / (sqrt(v') + eps)).
  * The update uses the unrounded binary32 m', v'; only the stored state is quantized.
  * ------------------------------------------------------------------------------------ */
 typedef struct {
@@ -302,11 +305,17 @@ static void update_element(int optim, const derived_scalars* d, float* p, float 
         pv = pv * d->decay;
         pv = pv - d->lr * s;
         *m = d->b2 * (*m) + d->omb2 * g;
-    } else { /* OR_MOMENTUM */
+    } else if (optim == OR_MOMENTUM) {
         if (d->wd != 0.0f) g = g + d->wd * pv;
         float m1 = d->b1 * (*m) + g;
         pv = pv - d->lr * m1;
         *m = m1;
+    } else { /* OR_RMSPROP: the state slot m holds the mean of squares */
+        if (d->wd != 0.0f) g = g + d->wd * pv;
+        float v1 = d->b1 * (*m) + (d->omb1 * g) * g;
+        float denom = sqrtf(v1) + d->eps;
+        pv = pv - d->lr * (g / denom);
+        *m = v1;
     }
     *p = pv;
 }
@@ -316,7 +325,7 @@ int oracle_step_blocks(int optim, int state_bits, float* p, const void* g, int g
                        const float* code2, int B, const oracle_hparams* hp, int t, int64_t b0,
                        int64_t b1)
 {
-    if (optim < OR_ADAMW || optim > OR_MOMENTUM || (state_bits != 8 && state_bits != 32)) return -1;
+    if (optim < OR_ADAMW || optim > OR_RMSPROP || (state_bits != 8 && state_bits != 32)) return -1;
     if (n < 0 || !valid_blocksize(B) || t < 1 || !hp) return -1;
     if (n == 0) return 0;
     int ns = n_states(optim);

@@ -24,6 +24,10 @@
  *  [ADAM]  D. Kingma, J. Ba, "Adam: A Method for Stochastic Optimization", Algorithm 1;
  *          I. Loshchilov, F. Hutter, "Decoupled Weight Decay Regularization", Algorithm 2.
  *  [LION]  X. Chen et al., "Symbolic Discovery of Optimization Algorithms", Algorithm 2 (Lion).
+ *  [RMSP]  T. Tieleman, G. Hinton, "Lecture 6.5 -- rmsprop: divide the gradient by a running
+ *          average of its recent magnitude", COURSERA: Neural Networks for Machine Learning,
+ *          2012; eps added outside the square root and weight decay added to the gradient, as
+ *          in torch.optim.RMSprop (no momentum, not centered).
  *  [QLORA] T. Dettmers et al., "QLoRA: Efficient Finetuning of Quantized LLMs", section 3
  *          (NormalFloat: quantiles of N(0,1), asymmetric 8+7 split with one shared zero).
  *
@@ -47,7 +51,7 @@ extern "C" {
 #endif
 
 /* optimizer ids and dtype ids used by the oracle (its own numbering) */
-enum { OR_ADAMW = 0, OR_ADAM = 1, OR_LION = 2, OR_MOMENTUM = 3 };
+enum { OR_ADAMW = 0, OR_ADAM = 1, OR_LION = 2, OR_MOMENTUM = 3, OR_RMSPROP = 4 };
 enum { OR_F32 = 0, OR_BF16 = 1 };
 
 typedef struct {

@@ -155,6 +155,74 @@ def test_lion_sign_update(oracle_mod):
     np.testing.assert_allclose(m, m64, rtol=1e-6, atol=1e-12)
 
 
+@pytest.mark.parametrize("wd", [0.0, 1e-2])
+def test_rmsprop_matches_torch(oracle_mod, wd):
+    """RMSprop (named by the page "bitsandbytes深度解析", section "优化器模块深度分析", as
+    RMSprop8bit) against torch.optim.RMSprop in float64: alpha in beta1, eps outside the root,
+    L2 weight decay, no momentum."""
+    n, steps, alpha = 3000, 8, 0.99
+    p0 = (np.random.default_rng(10).standard_normal(n) * 0.02).astype(np.float32)
+    grads = _grads(n, steps, 11)
+    p = p0.copy()
+    v = np.zeros(n, np.float32)
+    for t, g in enumerate(grads, 1):
+        oracle_mod.step_tensor("rmsprop", p, g, v, None, None, None, None, None, 2048, step=t,
+                               lr=1e-3, beta1=alpha, beta2=0.0, eps=1e-8, weight_decay=wd)
+    pt, st = _torch_run(torch.optim.RMSprop, p0, grads, lr=_f(1e-3), alpha=_f(alpha), eps=_f(1e-8),
+                        weight_decay=_f(wd), foreach=False)
+    # each step moves p by about lr/sqrt(1-alpha) = 10 lr at most
+    _close(p, pt, np.abs(p0) + 1e-2 * steps, rtol=1e-6)
+    _close(v, st["square_avg"].numpy(), np.max(v), rtol=2e-5)
+
+
+def test_rmsprop_first_step_closed_form(oracle_mod):
+    """P5-style closed form: from zero state v' = (1-alpha) g^2, so step 1 is
+    p - lr * g / (sqrt(1-alpha) |g| + eps)."""
+    n, alpha, lr, eps = 4096, 0.9, 1e-3, 1e-8
+    rng = np.random.default_rng(12)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    p, v = p0.copy(), np.zeros(n, np.float32)
+    oracle_mod.step_tensor("rmsprop", p, g, v, None, None, None, None, None, 256, step=1,
+                           lr=lr, beta1=alpha, beta2=0.0, eps=eps, weight_decay=0.0)
+    g64 = g.astype(np.float64)
+    oma = 1 - _f(alpha)
+    want = p0 - _f(lr) * g64 / (np.sqrt(oma) * np.abs(g64) + _f(eps))
+    _close(p, want, np.abs(p0) + 10 * lr, rtol=0)
+    _close(v, oma * g64 * g64, np.max(v), rtol=2e-6)
+
+
+def test_rmsprop_8bit_step_matches_torch(oracle_mod):
+    """8-bit RMSprop keeps its one state with the unsigned code: a step from a random 8-bit state
+    equals torch's RMSprop from the dequantized state, and the new state is the nearest code."""
+    n, B, alpha = 8192 + 5, 2048, 0.99
+    rng = np.random.default_rng(13)
+    code = oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    q = rng.integers(0, 256, n).astype(np.uint8)
+    a = rng.uniform(1e-8, 1e-6, nb).astype(np.float32)
+    v0 = _dequant(code, q, a, n, B)
+    p = p0.copy()
+    oracle_mod.step_tensor("rmsprop", p, g, q, None, a, None, code, None, B, step=4,
+                           lr=1e-3, beta1=alpha, beta2=0.0, eps=1e-8, weight_decay=0.0)
+    tp = torch.nn.Parameter(torch.from_numpy(p0.astype(np.float64)))
+    opt = torch.optim.RMSprop([tp], lr=_f(1e-3), alpha=_f(alpha), eps=_f(1e-8), foreach=False)
+    opt.state[tp] = {"step": torch.tensor(3.0), "square_avg": torch.from_numpy(v0.copy())}
+    tp.grad = torch.from_numpy(g.astype(np.float64))
+    opt.step()
+    _close(p, tp.detach().numpy(), np.abs(p0) + 1e-2, rtol=1e-6)
+    v1 = opt.state[tp]["square_avg"].numpy()
+    want_a = np.array([np.max(v1[i:i + B]) for i in range(0, n, B)])
+    np.testing.assert_allclose(a, want_a, rtol=1e-6)
+    xn = v1 / np.repeat(want_a, B)[:n]
+    qq, margin = _nearest_exact(code, xn)
+    far = margin > 1e-5 * np.maximum(np.abs(xn), 1e-7)
+    assert far.mean() > 0.99
+    np.testing.assert_array_equal(q[far], qq[far])
+
+
 # ----------------------------------------------------------------------- 8-bit state path
 def _dequant(code, q, absmax, n, B):
     return code[q].astype(np.float64) * np.repeat(absmax.astype(np.float64), B)[:n]
