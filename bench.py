@@ -45,6 +45,8 @@ WORKLOADS = {
                      (1e-4, 100.0)),
     "llama7b_momentum": ("llama7b", "momentum", 3, dict(lr=1e-2, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=0.0),
                          (1e-4, 100.0)),
+    "llama7b_rmsprop": ("llama7b", "rmsprop", 3, dict(lr=1e-3, beta1=0.99, beta2=0.0, eps=1e-8, weight_decay=0.0),
+                        (1e-4, 100.0)),
     # one decoder layer (202M params, ~3 GB): the size used for ncu captures
     "llama7b_layer_adamw": ("llama7b_layer", "adamw", 4,
                             dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01), (0.0, 1.0)),
@@ -234,7 +236,8 @@ def oracle_rate(shape: str, optim: str, hp: dict, elements8: int, threads: int, 
                     a1=None, a2=None)
 
     work = [(arrays(n8, 8), n8)] + ([(arrays(n32, 32), n32)] if n32 else [])
-    c1, c2 = oracle.code_dynamic_signed(), oracle.code_dynamic_unsigned()
+    c1 = oracle.code_dynamic_unsigned() if optim == "rmsprop" else oracle.code_dynamic_signed()
+    c2 = oracle.code_dynamic_unsigned()
     jobs = []
     for arrs, n in work:
         nb = (n + B - 1) // B

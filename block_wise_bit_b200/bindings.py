@@ -18,8 +18,8 @@ from . import build as _build
 
 OK, EINVAL, EUNSUPPORTED, ECUDA = 0, 1, 2, 3
 F32, BF16 = 0, 1
-ADAMW, ADAM, LION, MOMENTUM = 0, 1, 2, 3
-OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM}
+ADAMW, ADAM, LION, MOMENTUM, RMSPROP = 0, 1, 2, 3, 4
+OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM, "rmsprop": RMSPROP}
 CODE_DYNAMIC_SIGNED, CODE_DYNAMIC_UNSIGNED, CODE_NF4, CODE_LINEAR = 0, 1, 2, 3
 CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DYNAMIC_UNSIGNED,
               "nf4": CODE_NF4, "linear": CODE_LINEAR}

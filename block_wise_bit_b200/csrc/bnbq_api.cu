@@ -389,7 +389,7 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
                            const bnbq_hparams* hp, int step, const float* code1,
                            const float* code2, int blocksize, bnbq_stream_t stream)
 {
-    if (opt < BNBQ_ADAMW || opt > BNBQ_MOMENTUM) return fail(BNBQ_EINVAL, "unknown optimizer %d", (int)opt);
+    if (opt < BNBQ_ADAMW || opt > BNBQ_RMSPROP) return fail(BNBQ_EINVAL, "unknown optimizer %d", (int)opt);
     if (ntensors < 0 || ntensors > (1 << 20)) return fail(BNBQ_EINVAL, "ntensors %d out of [0, 2^20]", ntensors);
     if (ntensors > 0 && !list) return fail(BNBQ_EINVAL, "list is NULL");
     if (!hp) return fail(BNBQ_EINVAL, "hp is NULL");
@@ -401,6 +401,8 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
     const bool two = (opt == BNBQ_ADAMW || opt == BNBQ_ADAM);
     if (two && !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f && hp->beta2 >= 0.0f && hp->beta2 < 1.0f))
         return fail(BNBQ_EINVAL, "Adam betas must lie in [0, 1)");
+    if (opt == BNBQ_RMSPROP && !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f))
+        return fail(BNBQ_EINVAL, "RMSprop alpha (beta1) must lie in [0, 1)");
 
     std::vector<StepDesc> descs;
     descs.reserve(ntensors);

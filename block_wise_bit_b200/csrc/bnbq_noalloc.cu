@@ -66,7 +66,7 @@ extern "C" BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnb
                                                        const bnbq_hparams* hp, int step, const float* code1,
                                                        const float* code2, int blocksize, bnbq_stream_t stream)
 {
-    if (opt < BNBQ_ADAMW || opt > BNBQ_MOMENTUM) return fail(BNBQ_EINVAL, "unknown optimizer %d", (int)opt);
+    if (opt < BNBQ_ADAMW || opt > BNBQ_RMSPROP) return fail(BNBQ_EINVAL, "unknown optimizer %d", (int)opt);
     if (ntensors < 0) return fail(BNBQ_EINVAL, "ntensors %d < 0", ntensors);
     if (ntensors > 0 && !list) return fail(BNBQ_EINVAL, "list is NULL");
     if (!hp) return fail(BNBQ_EINVAL, "hp is NULL");
@@ -79,6 +79,8 @@ extern "C" BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnb
     const bool two = (opt == BNBQ_ADAMW || opt == BNBQ_ADAM);
     if (two && !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f && hp->beta2 >= 0.0f && hp->beta2 < 1.0f))
         return fail(BNBQ_EINVAL, "Adam betas must lie in [0, 1)");
+    if (opt == BNBQ_RMSPROP && !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f))
+        return fail(BNBQ_EINVAL, "RMSprop alpha (beta1) must lie in [0, 1)");
 
     std::lock_guard<std::mutex> lk(g_na_mu);  // one host staging array for all threads
     StepDesc* descs = g_na_host;

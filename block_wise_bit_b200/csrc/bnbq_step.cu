@@ -5,7 +5,7 @@
 // dynamic quantization while the update runs at 32-bit precision.  Per block this kernel
 //   loads p (fp32), g (fp32/bf16), the 8-bit codes and the block scales        (a4)
 //   dequantizes m = code1[q1]*a1 and v = code2[q2]*a2 from shared memory         (a4)
-//   applies the fp32 AdamW / Adam / Lion / momentum update and stores p at once   (a5)
+//   applies the fp32 AdamW / Adam / Lion / momentum / RMSprop update, stores p    (a5)
 //   reduces the new block absmax of each state across the block's thread group     (a6)
 //   requantizes each state against its new absmax (nearest code) and stores it     (a7)
 // Tensors that keep 32-bit state (fewer than 4096 elements, and embedding tables: page
@@ -107,11 +107,18 @@ __device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, f
         p = mul2(p, k.decay);
         p = add2(p, mul2(k.nlr, sg));
         m = add2(mul2(k.b2, m), mul2(k.omb2, g));
-    } else {  // momentum SGD, dampening 0
+    } else if constexpr (OPT == BNBQ_MOMENTUM) {  // dampening 0
         if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
         const float2 m1 = add2(mul2(k.b1, m), g);
         p = add2(p, mul2(k.nlr, m1));
         m = m1;
+    } else {  // RMSprop: the one state (m) is the running mean of squares, b1 = alpha
+        if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
+        const float2 v1 = add2(mul2(k.b1, m), mul2(mul2(k.omb1, g), g));
+        const float2 den = add2(make_float2(__fsqrt_rn(v1.x), __fsqrt_rn(v1.y)), k.eps);
+        const float2 u = make_float2(__fdiv_rn(g.x, den.x), __fdiv_rn(g.y, den.y));
+        p = add2(p, mul2(k.nlr, u));
+        m = v1;
     }
 }
 
@@ -583,6 +590,7 @@ bnbq_status launch_step(bnbq_optim opt, const StepDesc* d_table, int ntensors, i
         case BNBQ_ADAM: return launch_step_o<BNBQ_ADAM>(d_table, ntensors, total_blocks, sc, code1, code2, B, s);
         case BNBQ_LION: return launch_step_o<BNBQ_LION>(d_table, ntensors, total_blocks, sc, code1, code2, B, s);
         case BNBQ_MOMENTUM: return launch_step_o<BNBQ_MOMENTUM>(d_table, ntensors, total_blocks, sc, code1, code2, B, s);
+        case BNBQ_RMSPROP: return launch_step_o<BNBQ_RMSPROP>(d_table, ntensors, total_blocks, sc, code1, code2, B, s);
         default: return fail(BNBQ_EINVAL, "unknown optimizer %d", (int)opt);
     }
 }

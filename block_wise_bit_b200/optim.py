@@ -74,6 +74,11 @@ class Optimizer8bit(torch.optim.Optimizer):
     def two_states(self) -> bool:
         return self._KIND in ("adamw", "adam")
 
+    @property
+    def code1_kind(self) -> str:
+        """Codebook of the first state: signed, except RMSprop's non-negative mean of squares."""
+        return "dynamic_unsigned" if self._KIND == "rmsprop" else "dynamic_signed"
+
     def override_32bit(self, param: torch.Tensor) -> None:
         """Keep ``param``'s state in 32 bits (e.g. an embedding table)."""
         self._force32.add(id(param))
@@ -94,7 +99,7 @@ class Optimizer8bit(torch.optim.Optimizer):
             if not params:
                 continue
             dev = params[0].device
-            code1 = device_codebook("dynamic_signed", dev)
+            code1 = device_codebook(self.code1_kind, dev)
             code2 = device_codebook("dynamic_unsigned", dev) if self.two_states else None
             entries: List[B.TensorState] = []
             for p in params:
@@ -145,6 +150,15 @@ class SGD8bit(Optimizer8bit):
         super().__init__(params, lr, (momentum, 0.0), 0.0, weight_decay, **kw)
 
 
+class RMSprop8bit(Optimizer8bit):
+    """RMSprop without momentum (torch.optim.RMSprop's default form); ``alpha`` is passed to the
+    kernel as beta1 and the one state uses the unsigned dynamic code."""
+    _KIND = "rmsprop"
+
+    def __init__(self, params, lr=1e-2, alpha=0.99, eps=1e-8, weight_decay=0.0, **kw):
+        super().__init__(params, lr, (alpha, 0.0), eps, weight_decay, **kw)
+
+
 class FlatStateList:
     """A whole parameter list laid out in flat device buffers (see ``workloads.Layout``), with
     its 8-bit / 32-bit state and the tensor list packed once for repeated steps."""
@@ -154,7 +168,7 @@ class FlatStateList:
         self.optim = optim
         self.two = optim in ("adamw", "adam")
         self.device = torch.device(device)
-        self.code1 = device_codebook("dynamic_signed", self.device)
+        self.code1 = device_codebook("dynamic_unsigned" if optim == "rmsprop" else "dynamic_signed", self.device)
         self.code2 = device_codebook("dynamic_unsigned", self.device) if self.two else None
         lay = layout
         self.p = torch.empty(lay.total, dtype=torch.float32, device=self.device)

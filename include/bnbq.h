@@ -56,8 +56,9 @@ typedef enum { BNBQ_F32 = 0, BNBQ_BF16 = 1 } bnbq_dtype;
 typedef enum {
     BNBQ_ADAMW = 0,   /* Adam with decoupled weight decay (two states: m signed, v unsigned) */
     BNBQ_ADAM = 1,    /* Adam, weight decay added to the gradient (two states) */
-    BNBQ_LION = 2,    /* Lion: one signed state */
-    BNBQ_MOMENTUM = 3 /* SGD with momentum, dampening 0: one signed state */
+    BNBQ_LION = 2,     /* Lion: one signed state */
+    BNBQ_MOMENTUM = 3, /* SGD with momentum, dampening 0: one signed state */
+    BNBQ_RMSPROP = 4   /* RMSprop: one state, the running mean of squares (unsigned code) */
 } bnbq_optim;
 
 typedef enum {
@@ -113,7 +114,8 @@ typedef struct {
 } bnbq_tensor;
 
 /* Hyper-parameters as torch.optim names them.  Momentum SGD reads beta1 as its momentum;
- * Lion reads beta1 (update interpolation) and beta2 (state decay). */
+ * Lion reads beta1 (update interpolation) and beta2 (state decay); RMSprop reads beta1 as its
+ * smoothing constant alpha. */
 typedef struct {
     float lr, beta1, beta2, eps, weight_decay;
 } bnbq_hparams;
@@ -126,9 +128,11 @@ typedef struct {
  * "Py之bitsandbytes…详细攻略", section "如果需要高精度的参数").
  *   opt         bnbq_optim
  *   list        host array of ntensors descriptors (0 <= ntensors <= 1<<20)
- *   hp          host pointer; all values finite; for Adam/AdamW 0 <= beta1, beta2 < 1
+ *   hp          host pointer; all values finite; for Adam/AdamW 0 <= beta1, beta2 < 1; for
+ *               RMSprop 0 <= beta1 < 1
  *   step        t >= 1, the 1-based step number shared by all tensors (Adam bias correction)
- *   code1       device, 256 fp32: signed code for state1 (needed if any tensor is 8-bit)
+ *   code1       device, 256 fp32: code for state1 (needed if any tensor is 8-bit): the signed
+ *               code, or for RMSprop the unsigned one
  *   code2       device, 256 fp32: unsigned code for Adam/AdamW state2 (else may be NULL)
  *   blocksize   256, 2048 or 4096
  * Per element, in binary32 with every operation rounded on its own:
@@ -137,6 +141,10 @@ typedef struct {
  *   Adam:  g = g + wd*p (if wd != 0), then AdamW's rule without the p*(1-lr*wd) factor
  *   Lion:  c = b1*m + (1-b1)*g; p = p*(1-lr*wd) - lr*sign(c); m = b2*m + (1-b2)*g
  *   Momentum: g = g + wd*p (if wd != 0); m = b1*m + g; p = p - lr*m
+ *   RMSprop: g = g + wd*p (if wd != 0); v = b1*v + ((1-b1)*g)*g; p = p - lr * (g / (sqrt(v) + eps))
+ *          (T. Tieleman, G. Hinton, "Lecture 6.5 -- rmsprop", 2012; eps outside the root, as in
+ *          torch.optim.RMSprop without momentum; the pages name RMSprop8bit in
+ *          "bitsandbytes深度解析", section "优化器模块深度分析")
  * (scalar factors such as 1-b1, lr/(1-b1^t) are formed in double on the host and rounded once.)
  * For 8-bit state the old state is code[q]*absmax[b]; after the update each block gets a new
  * absmax = max|state| and the state is requantized by the nearest-code rule above.

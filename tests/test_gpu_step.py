@@ -6,7 +6,7 @@
   step.  Plus standalone quantize / dequantize of the same tensor.
 * Every optimizer x blocksize x gradient dtype on a small multi-tensor list with ragged tails
   and 32-bit-state members, from a synthetic non-zero state, several steps.
-* GPT-2-1.5B AdamW and 7B Llama AdamW / Lion / momentum lists at full size, stepped whole by
+* GPT-2-1.5B AdamW and 7B Llama AdamW / Lion / momentum / RMSprop lists at full size, stepped whole by
   one launch per step (the benchmark's launch configuration); sampled tensors / block ranges are
   recomputed by the oracle from the same seeded inputs along their own trajectory.
 Bar: p within 1e-6 relative or 1e-9 absolute; codes equal except within 2 ulp of a decision
@@ -30,6 +30,7 @@ HP = {
     "adam": dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
     "lion": dict(lr=1e-4, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=0.1),
     "momentum": dict(lr=1e-2, beta1=0.9, beta2=0.0, eps=0.0, weight_decay=0.0),
+    "rmsprop": dict(lr=1e-3, beta1=0.99, beta2=0.0, eps=1e-8, weight_decay=0.01),
 }
 REPORT = []
 
@@ -46,8 +47,10 @@ def _cuda():
         print(line)
 
 
-def _codes():
-    return bq.bnbq_codebook("dynamic_signed"), bq.bnbq_codebook("dynamic_unsigned")
+def _codes(optim="adamw"):
+    """(code1, code2): the first state's code is signed, except RMSprop's mean of squares."""
+    first = "dynamic_unsigned" if optim == "rmsprop" else "dynamic_signed"
+    return bq.bnbq_codebook(first), bq.bnbq_codebook("dynamic_unsigned")
 
 
 class HostTensor:
@@ -132,7 +135,7 @@ def _small_list(optim, B, g_dtype, seed, codes=None):
     """Tensors of SIZES (policy: < 4096 -> 32-bit) plus one large tensor forced to 32-bit, with
     a synthetic non-zero state."""
     two = optim in ("adamw", "adam")
-    c1, c2 = codes if codes is not None else _codes()
+    c1, c2 = codes if codes is not None else _codes(optim)
     out = []
     for i, n in enumerate(SIZES + [30000]):
         bits = 32 if (n < 4096 or i == len(SIZES)) else 8
@@ -148,15 +151,19 @@ def _small_list(optim, B, g_dtype, seed, codes=None):
             a2 = W.log_uniform(nb, 1e-8, 1e-5, DEV, "small", seed, i, "a2") if two else None
             if optim == "momentum":
                 a1 = W.log_uniform(nb, 1e-3, 1e-1, DEV, "small", seed, i, "a1m")
+            if optim == "rmsprop":  # mean of squares
+                a1 = W.log_uniform(nb, 1e-8, 1e-5, DEV, "small", seed, i, "a1r")
         else:
             s1 = W.normal(n, 1e-3, DEV, "small", seed, i, "m")
+            if optim == "rmsprop":
+                s1.square_()
             s2 = W.normal(n, 1e-3, DEV, "small", seed, i, "v").square_() if two else None
             a1 = a2 = None
         out.append(bq.TensorState(p, g, s1, s2, a1, a2))
     return out, c1, c2
 
 
-@pytest.mark.parametrize("optim", ["adamw", "adam", "lion", "momentum"])
+@pytest.mark.parametrize("optim", ["adamw", "adam", "lion", "momentum", "rmsprop"])
 @pytest.mark.parametrize("B", [256, 2048, 4096])
 @pytest.mark.parametrize("g_dtype", [torch.float32, torch.bfloat16])
 def test_small_list_all_optimizers(optim, B, g_dtype):
@@ -308,7 +315,7 @@ def _full_size_run(shape, optim, seed, steps, picks_fn, g_outlier=(0.0, 1.0)):
     fl = O.FlatStateList(lay, optim, DEV, g_dtype=torch.bfloat16)
     for i, spec in enumerate(lay.specs):
         fl.entries[i].p.copy_(W.normal(spec.numel, 0.02, DEV, shape, seed, i, "p"))
-    c1, c2 = _codes()
+    c1, c2 = _codes(optim)
     two = optim in ("adamw", "adam")
     ranges = _sample_ranges(lay, B, picks_fn(lay))
     hosts = [HostTensor(_slice_state(fl, i, b0, b1)) for (i, b0, b1) in ranges]
@@ -349,8 +356,8 @@ def test_gpt2_1p5b_adamw_full_size():
     _full_size_run("gpt2_1p5b", "adamw", 2, 6, _gpt2_picks)
 
 
-@pytest.mark.parametrize("optim", ["lion", "momentum"])
-def test_llama7b_lion_momentum_full_size(optim):
+@pytest.mark.parametrize("optim", ["lion", "momentum", "rmsprop"])
+def test_llama7b_one_state_full_size(optim):
     _full_size_run("llama7b", optim, 3, 2, _llama_picks, g_outlier=(1e-4, 100.0))
 
 
