@@ -69,6 +69,12 @@ def lib():
             L.oracle_step_blocks.argtypes = [i32, i32, vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, i32,
                                              ctypes.POINTER(_HP), i32, i64, i64]
             L.oracle_step_blocks.restype = i32
+            L.oracle_absmax_mean.argtypes = [vp, i64]
+            L.oracle_absmax_mean.restype = ctypes.c_float
+            L.oracle_nest_absmax.argtypes = [vp, i64, vp, vp, vp, vp]
+            L.oracle_nest_absmax.restype = i32
+            L.oracle_unnest_absmax.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp]
+            L.oracle_unnest_absmax.restype = i32
             _lib = L
     return _lib
 
@@ -156,6 +162,48 @@ def dequantize_blockwise(code: np.ndarray, q: np.ndarray, absmax: np.ndarray, n:
     if rc != 0:
         raise ValueError("oracle_dequantize_blockwise rejected its arguments")
     return y
+
+
+# ---------------------------------------------------------------- nested quantization of scales
+NEST_B = 256
+NEST_CHUNK = 4096
+
+
+def absmax_mean(absmax: np.ndarray) -> np.float32:
+    absmax = _f32(absmax)
+    return np.float32(lib().oracle_absmax_mean(_ptr(absmax), absmax.size))
+
+
+def nest_absmax(absmax: np.ndarray, code2: np.ndarray):
+    """Return (qabs uint8[nb], absmax2 float32[ceil(nb/256)], offset float32)."""
+    absmax = _f32(absmax)
+    code2 = _f32(code2)
+    nb = absmax.size
+    qabs = np.zeros(nb, np.uint8)
+    absmax2 = np.zeros((nb + NEST_B - 1) // NEST_B, np.float32)
+    off = np.zeros(1, np.float32)
+    rc = lib().oracle_nest_absmax(_ptr(absmax), nb, _ptr(code2), _ptr(qabs), _ptr(absmax2), _ptr(off))
+    if rc != 0:
+        raise ValueError("oracle_nest_absmax rejected its arguments")
+    return qabs, absmax2, np.float32(off[0])
+
+
+def unnest_absmax(qabs: np.ndarray, absmax2: np.ndarray, offset, code2: np.ndarray) -> np.ndarray:
+    qabs = np.ascontiguousarray(qabs, dtype=np.uint8)
+    absmax2 = _f32(absmax2)
+    code2 = _f32(code2)
+    out = np.zeros(qabs.size, np.float32)
+    rc = lib().oracle_unnest_absmax(_ptr(qabs), _ptr(absmax2), ctypes.c_float(float(offset)), _ptr(code2),
+                                    qabs.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_unnest_absmax rejected its arguments")
+    return out
+
+
+def dequantize_blockwise_nested(code: np.ndarray, q: np.ndarray, qabs: np.ndarray, absmax2: np.ndarray, offset,
+                                code2: np.ndarray, n: int, blocksize: int, out_bf16: bool = False) -> np.ndarray:
+    """Dequantize with block scales rebuilt from their nested quantization."""
+    return dequantize_blockwise(code, q, unnest_absmax(qabs, absmax2, offset, code2), n, blocksize, out_bf16)
 
 
 # ---------------------------------------------------------------- optimizer step

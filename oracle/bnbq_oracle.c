@@ -9,6 +9,7 @@
 
 #include <math.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ------------------------------------------------------------------------------------
@@ -167,7 +168,7 @@ static float load_value(const void* x, int dtype, int64_t i)
     return ((const float*)x)[i];
 }
 
-static int valid_blocksize(int B) { return B == 256 || B == 2048 || B == 4096; }
+static int valid_blocksize(int B) { return B == 64 || B == 128 || B == 256 || B == 2048 || B == 4096; }
 
 /* ------------------------------------------------------------------------------------
  * Block-wise quantization [BWQ]: the tensor is cut into blocks of B consecutive elements
@@ -238,6 +239,56 @@ int oracle_dequantize_blockwise(const float* code, int K, const uint8_t* q, cons
         else
             ((float*)y)[e] = v;
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Nested (double) quantization of the block scales [NEST]: the fp32 absmax array of an
+ * already quantized tensor is itself quantized.  Following [QLORA] (section 3, "Double
+ * Quantization"): the scales are centred by their mean (they are all >= 0, the code is
+ * signed) and quantized block-wise to 8 bits in blocks of 256 with the signed dynamic code.
+ * Reconstruction: a_i = code2[qabs_i] * absmax2[i / 256] + offset (two roundings).
+ * READING: the mean's summation order is not given anywhere; it is fixed here as a double
+ * sum over chunks of 4096 consecutive scales (each chunk summed in index order, the chunk
+ * sums added in index order), divided by nb in double and rounded once to float.
+ * ------------------------------------------------------------------------------------ */
+float oracle_absmax_mean(const float* absmax, int64_t nb)
+{
+    if (nb <= 0) return 0.0f;
+    double total = 0.0;
+    for (int64_t c = 0; c < nb; c += ORACLE_NEST_CHUNK) {
+        int64_t end = (c + ORACLE_NEST_CHUNK < nb) ? c + ORACLE_NEST_CHUNK : nb;
+        double s = 0.0;
+        for (int64_t i = c; i < end; i++) s += (double)absmax[i];
+        total += s;
+    }
+    return (float)(total / (double)nb);
+}
+
+int oracle_nest_absmax(const float* absmax, int64_t nb, const float* code2, uint8_t* qabs,
+                       float* absmax2, float* offset)
+{
+    if (nb < 0 || !code2 || !offset) return -1;
+    *offset = 0.0f;
+    if (nb == 0) return 0;
+    if (!absmax || !qabs || !absmax2) return -1;
+    float mean = oracle_absmax_mean(absmax, nb);
+    float* centred = (float*)malloc((size_t)nb * sizeof(float));
+    if (!centred) return -1;
+    for (int64_t i = 0; i < nb; i++) centred[i] = absmax[i] - mean;
+    int rc = oracle_quantize_blockwise(code2, 256, centred, OR_F32, nb, ORACLE_NEST_B, absmax2, qabs);
+    free(centred);
+    *offset = mean;
+    return rc;
+}
+
+int oracle_unnest_absmax(const uint8_t* qabs, const float* absmax2, float offset, const float* code2,
+                         int64_t nb, float* out)
+{
+    if (nb < 0 || !code2) return -1;
+    if (nb == 0) return 0;
+    if (!qabs || !absmax2 || !out) return -1;
+    for (int64_t i = 0; i < nb; i++) out[i] = code2[qabs[i]] * absmax2[i / ORACLE_NEST_B] + offset;
     return 0;
 }
 

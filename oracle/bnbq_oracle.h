@@ -29,7 +29,11 @@
  *          2012; eps added outside the square root and weight decay added to the gradient, as
  *          in torch.optim.RMSprop (no momentum, not centered).
  *  [QLORA] T. Dettmers et al., "QLoRA: Efficient Finetuning of Quantized LLMs", section 3
- *          (NormalFloat: quantiles of N(0,1), asymmetric 8+7 split with one shared zero).
+ *          (NormalFloat: quantiles of N(0,1), asymmetric 8+7 split with one shared zero;
+ *          Double Quantization: the constants quantized again, 8-bit, blocks of 256, centred).
+ *  [NEST]  page "Bitsandbytes" (transformers docs, Turkish), section "İç içe nicelleştirme"
+ *          (nested quantization: a second quantization of the already quantized weights'
+ *          constants, about 0.4 bit per parameter saved).
  *
  * Floating point: IEEE binary32, round to nearest even, every operation rounded on its own
  * (built with -ffp-contract=off, no -ffast-math), division and sqrtf correctly rounded,
@@ -86,6 +90,20 @@ int oracle_quantize_blockwise(const float* code, int K, const void* x, int x_dty
 /* y_i = code[q_i] * absmax_b, written as float (OR_F32) or bf16 bits (OR_BF16). */
 int oracle_dequantize_blockwise(const float* code, int K, const uint8_t* q, const float* absmax,
                                 int64_t n, int B, void* y, int y_dtype);
+
+/*
+ * Nested (double) quantization of a block-scale array absmax[nb] [NEST]: offset = mean of the
+ * scales (double sum over chunks of ORACLE_NEST_CHUNK, rounded once), then the centred scales
+ * absmax_i - offset are quantized block-wise (blocks of ORACLE_NEST_B) with the 256-entry code2:
+ * qabs[nb], absmax2[ceil(nb/ORACLE_NEST_B)].  Unnest rebuilds code2[qabs_i]*absmax2[i/256]+offset.
+ */
+#define ORACLE_NEST_B 256
+#define ORACLE_NEST_CHUNK 4096
+float oracle_absmax_mean(const float* absmax, int64_t nb);
+int oracle_nest_absmax(const float* absmax, int64_t nb, const float* code2, uint8_t* qabs,
+                       float* absmax2, float* offset);
+int oracle_unnest_absmax(const uint8_t* qabs, const float* absmax2, float offset, const float* code2,
+                         int64_t nb, float* out);
 
 /*
  * One optimizer step on one tensor (t >= 1 is the step number, shared by all tensors).

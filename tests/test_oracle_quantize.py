@@ -94,7 +94,7 @@ def _blocks(x, B):
 
 
 @pytest.mark.parametrize("name", ["signed", "unsigned", "nf4", "linear"])
-@pytest.mark.parametrize("B", [256, 2048, 4096])
+@pytest.mark.parametrize("B", [64, 128, 256, 2048, 4096])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_quantize_blockwise_matches_bruteforce(oracle_mod, name, B, bf16):
     code = _codes(oracle_mod)[name]
