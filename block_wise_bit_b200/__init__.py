@@ -6,10 +6,12 @@ RMSprop step.  ``bindings`` is its ctypes marshalling layer (same names as the C
 ``optim`` holds the launcher policy (which tensors keep 32-bit state) and torch.optim-style
 front ends; ``workloads`` describes seeded synthetic parameter lists.
 """
-from .bindings import (BnbqError, TensorState, bnbq_check_codebook, bnbq_codebook, bnbq_dequantize_blockwise,
-                       bnbq_device_flags, bnbq_last_error, bnbq_quantize_blockwise, bnbq_release, bnbq_step_8bit,
-                       bnbq_version, lib, pack_tensor_list)
+from .bindings import (BnbqError, TensorState, bnbq_check_codebook, bnbq_codebook, bnbq_dequantize_absmax_nested,
+                       bnbq_dequantize_blockwise, bnbq_dequantize_blockwise_nested, bnbq_device_flags,
+                       bnbq_last_error, bnbq_quantize_absmax_nested, bnbq_quantize_blockwise, bnbq_release,
+                       bnbq_step_8bit, bnbq_version, lib, pack_tensor_list)
 
-__all__ = ["BnbqError", "TensorState", "bnbq_check_codebook", "bnbq_codebook", "bnbq_dequantize_blockwise",
-           "bnbq_device_flags", "bnbq_last_error", "bnbq_quantize_blockwise", "bnbq_release", "bnbq_step_8bit",
+__all__ = ["BnbqError", "TensorState", "bnbq_check_codebook", "bnbq_codebook", "bnbq_dequantize_absmax_nested",
+           "bnbq_dequantize_blockwise", "bnbq_dequantize_blockwise_nested", "bnbq_device_flags", "bnbq_last_error",
+           "bnbq_quantize_absmax_nested", "bnbq_quantize_blockwise", "bnbq_release", "bnbq_step_8bit",
            "bnbq_version", "lib", "pack_tensor_list"]

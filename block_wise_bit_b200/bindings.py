@@ -26,7 +26,8 @@ CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DY
 FLAG_BAD_CODE, FLAG_NONFINITE = 0x1, 0x2
 
 EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_step_8bit_noalloc",
-            "bnbq_codebook",
+            "bnbq_nested_workspace_bytes", "bnbq_quantize_absmax_nested", "bnbq_dequantize_absmax_nested",
+            "bnbq_dequantize_blockwise_nested", "bnbq_codebook",
             "bnbq_code_size", "bnbq_check_codebook", "bnbq_device_flags", "bnbq_last_error", "bnbq_release",
             "bnbq_version"]
 
@@ -79,6 +80,14 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
                                      i32, vp]
         L.bnbq_step_8bit_noalloc.argtypes = L.bnbq_step_8bit.argtypes
         L.bnbq_step_8bit_noalloc.restype = i32
+        L.bnbq_nested_workspace_bytes.argtypes = [i64]
+        L.bnbq_nested_workspace_bytes.restype = i64
+        L.bnbq_quantize_absmax_nested.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp]
+        L.bnbq_quantize_absmax_nested.restype = i32
+        L.bnbq_dequantize_absmax_nested.argtypes = [vp, vp, vp, vp, i64, vp, vp]
+        L.bnbq_dequantize_absmax_nested.restype = i32
+        L.bnbq_dequantize_blockwise_nested.argtypes = [vp, i32, vp, vp, vp, vp, vp, i64, i32, vp, i32, vp]
+        L.bnbq_dequantize_blockwise_nested.restype = i32
         for f in ("bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit",
                   "bnbq_check_codebook", "bnbq_device_flags"):
             getattr(L, f).restype = i32
@@ -169,6 +178,53 @@ def bnbq_dequantize_blockwise(code: torch.Tensor, q: torch.Tensor, absmax: torch
     _check(lib().bnbq_dequantize_blockwise(_dev(code, "code"), code.numel(), _dev(q, "q") if n else None,
                                            _dev(absmax, "absmax") if n else None, n, blocksize,
                                            _dev(out, "out") if n else None, _dtype_id(out), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------------- nested block scales
+NEST_BLOCK = 256
+
+
+def bnbq_quantize_absmax_nested(code2: torch.Tensor, absmax: torch.Tensor, stream=None):
+    """Nested quantization of a block-scale array: returns (qabs uint8[nb], absmax2 float32
+    [ceil(nb/256)], offset float32[1]), all on absmax's device.  The workspace is a torch
+    allocation made here."""
+    nb = absmax.numel()
+    dev = absmax.device
+    qabs = torch.empty(nb, dtype=torch.uint8, device=dev)
+    absmax2 = torch.empty((nb + NEST_BLOCK - 1) // NEST_BLOCK, dtype=torch.float32, device=dev)
+    offset = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, lib().bnbq_nested_workspace_bytes(nb)), dtype=torch.uint8, device=dev)
+    _check(lib().bnbq_quantize_absmax_nested(_dev(absmax, "absmax") if nb else None, nb, _dev(code2, "code2"),
+                                             _dev(qabs, "qabs") if nb else None,
+                                             _dev(absmax2, "absmax2") if nb else None, _dev(offset, "offset"),
+                                             _dev(ws, "workspace"), _stream(stream)))
+    return qabs, absmax2, offset
+
+
+def bnbq_dequantize_absmax_nested(code2: torch.Tensor, qabs: torch.Tensor, absmax2: torch.Tensor,
+                                  offset: torch.Tensor, stream=None) -> torch.Tensor:
+    nb = qabs.numel()
+    out = torch.empty(nb, dtype=torch.float32, device=qabs.device)
+    if nb:
+        _check(lib().bnbq_dequantize_absmax_nested(_dev(qabs, "qabs"), _dev(absmax2, "absmax2"),
+                                                   _dev(offset, "offset"), _dev(code2, "code2"), nb,
+                                                   _dev(out, "absmax_out"), _stream(stream)))
+    return out
+
+
+def bnbq_dequantize_blockwise_nested(code: torch.Tensor, q: torch.Tensor, qabs: torch.Tensor, absmax2: torch.Tensor,
+                                     offset: torch.Tensor, code2: torch.Tensor, n: int, blocksize: int = 64,
+                                     out_dtype=torch.float32, out: Optional[torch.Tensor] = None,
+                                     stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(n, dtype=out_dtype, device=q.device)
+    _check(lib().bnbq_dequantize_blockwise_nested(_dev(code, "code"), code.numel(), _dev(q, "q") if n else None,
+                                                  _dev(qabs, "qabs") if n else None,
+                                                  _dev(absmax2, "absmax2") if n else None,
+                                                  _dev(offset, "offset") if n else None, _dev(code2, "code2"), n,
+                                                  blocksize, _dev(out, "out") if n else None, _dtype_id(out),
+                                                  _stream(stream)))
     return out
 
 

@@ -96,6 +96,7 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool valid_blocksize(int B) { return B == 256 || B == 2048 || B == 4096; }
+bool valid_q_blocksize(int B) { return B == 64 || B == 128 || valid_blocksize(B); }
 bool valid_dtype(int d) { return d == BNBQ_F32 || d == BNBQ_BF16; }
 uintptr_t dtype_align(int d) { return d == BNBQ_BF16 ? 8 : 16; }
 
@@ -105,7 +106,7 @@ bnbq_status check_common(const float* code, int K, int64_t n, int B)
     if (K != 256 && K != 16) return fail(BNBQ_EINVAL, "code_size %d not in {16, 256}", K);
     if (!aligned(code, 4)) return fail(BNBQ_EINVAL, "code not 4-byte aligned");
     if (n < 0) return fail(BNBQ_EINVAL, "n = %lld < 0", (long long)n);
-    if (!valid_blocksize(B)) return fail(BNBQ_EINVAL, "blocksize %d not in {256, 2048, 4096}", B);
+    if (!valid_q_blocksize(B)) return fail(BNBQ_EINVAL, "blocksize %d not in {64, 128, 256, 2048, 4096}", B);
     return BNBQ_OK;
 }
 

@@ -26,6 +26,23 @@ bnbq_status launch_quantize(const float* code, int K, const void* A, bnbq_dtype 
 bnbq_status launch_dequantize(const float* code, int K, const uint8_t* q, const float* absmax,
                               int64_t n, int B, void* out, bnbq_dtype dt, cudaStream_t s);
 
+// Nested quantization of block scales: blocks of kNestBlock scales, the mean summed in double
+// over chunks of kNestChunk scales.
+constexpr int kNestBlock = 256;
+constexpr int kNestChunk = 4096;
+// absmax2/qabs <- block-wise quantization of a[i] - *center (fp32, blocks of kNestBlock).
+bnbq_status launch_quantize_centred(const float* code2, const float* a, int64_t nb, const float* center,
+                                    float* absmax2, uint8_t* qabs, cudaStream_t s);
+// Dequantize with block scales code2[qabs_b] * absmax2[b / kNestBlock] + *center.
+bnbq_status launch_dequantize_nested(const float* code, int K, const uint8_t* q, const uint8_t* qabs,
+                                     const float* absmax2, const float* center, const float* code2, int64_t n,
+                                     int B, void* out, bnbq_dtype dt, cudaStream_t s);
+// *center <- mean of a[0..nb) (double chunk sums into work[ceil(nb/kNestChunk)], rounded once).
+bnbq_status launch_absmax_mean(const float* a, int64_t nb, double* work, float* center, cudaStream_t s);
+// out[i] <- code2[qabs_i] * absmax2[i / kNestBlock] + *center.
+bnbq_status launch_unnest(const uint8_t* qabs, const float* absmax2, const float* center, const float* code2,
+                          int64_t nb, float* out, cudaStream_t s);
+
 // One entry of the device descriptor table used by the step kernel (64 bytes).
 struct alignas(16) StepDesc {
     float* p;

@@ -128,10 +128,12 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
     }
 }
 
-template <int B, bool BF16, int K, int MODE>
+// CENTER: quantize A[i] - *center (one binary32 subtraction; fp32 input), the centred block
+// scales of nested quantization.
+template <int B, bool BF16, int K, int MODE, bool CENTER>
 __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
                                               float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
-                                              unsigned* flags)
+                                              unsigned* flags, const float* __restrict__ center)
 {
     using Geo = QGeom<B>;
     constexpr int G = Geo::G;
@@ -140,6 +142,7 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
     const int lane = threadIdx.x & 31;
     const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
     const int64_t nb = (n + B - 1) / B;
+    const float off = CENTER ? __ldg(center) : 0.0f;
     int parity = 0;
 
     for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb; b += (int64_t)gridDim.x * Geo::kGroups) {
@@ -147,6 +150,13 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
         float v[4][4];
 #pragma unroll
         for (int j = 0; j < 4; j++) load_chunk<BF16>(A, base + 4 * (j * G + tg), n, v[j]);
+        if constexpr (CENTER) {
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    if (base + 4 * (j * G + tg) + i < n) v[j][i] = __fsub_rn(v[j][i], off);
+        }
 
         float m = 0.0f;
 #pragma unroll
@@ -178,10 +188,11 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
     }
 }
 
-template <int B, bool BF16, int K>
+template <int B, bool BF16, int K, bool CENTER>
 __global__ void __launch_bounds__(kQThreads, 2)
 quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
-                float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags)
+                float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags,
+                const float* __restrict__ center)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     CodeSmem& cs = *reinterpret_cast<CodeSmem*>(smem_raw);
@@ -189,23 +200,42 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     bool fast, general;
     if (!stage_one_code(cs, code, K, true, fast, general, flags)) return;
     if (general)
-        quantize_loop<B, BF16, K, kSearchGeneral>(cs, fast, A, n, absmax, out, red, flags);
+        quantize_loop<B, BF16, K, kSearchGeneral, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
     else if (cs.code[0] >= 0.0f)  // every code >= 0
-        quantize_loop<B, BF16, K, kSearchNonNeg>(cs, fast, A, n, absmax, out, red, flags);
+        quantize_loop<B, BF16, K, kSearchNonNeg, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
     else
-        quantize_loop<B, BF16, K, kSearchSigned>(cs, fast, A, n, absmax, out, red, flags);
+        quantize_loop<B, BF16, K, kSearchSigned, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
 }
 
 // Dequantize: flat grid over 4-element chunks; each thread takes 4 chunks per pass.
-template <int K, bool BF16OUT>
+// NESTED: the block scales are rebuilt from their nested quantization,
+// A_b = code2[qabs_b] * absmax2[b / 256] + *center (two roundings), instead of read from absmax.
+struct NestedScales {
+    const uint8_t* qabs;
+    const float* absmax2;
+    const float* center;
+    const float* code2;
+};
+
+template <int K, bool BF16OUT, bool NESTED>
 __global__ void __launch_bounds__(256)
 dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
                   const float* __restrict__ absmax, int64_t n, int log2B, void* __restrict__ out,
-                  unsigned* flags)
+                  unsigned* flags, NestedScales ns)
 {
-    __shared__ CodeSmem cs;
-    bool fast, general;
-    if (!stage_one_code(cs, code, K, false, fast, general, flags)) return;
+    __shared__ float code_s[NESTED ? 2 : 1][256];
+    __shared__ float mid_s[NESTED ? 2 : 1][256];
+    stage_codes(code_s[0], code, K);
+    if constexpr (NESTED) stage_codes(code_s[NESTED ? 1 : 0], ns.code2, 256);
+    __syncthreads();
+    bool bad = false, tiny = false;
+    stage_midpoints(code_s[0], mid_s[0], K, bad, tiny);
+    if constexpr (NESTED) stage_midpoints(code_s[NESTED ? 1 : 0], mid_s[NESTED ? 1 : 0], 256, bad, tiny);
+    if (__syncthreads_or(bad)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
+        return;
+    }
+    const float off = NESTED ? __ldg(ns.center) : 0.0f;
 
     const int64_t nchunks = (n + 3) / 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -234,7 +264,12 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
                         if (e + 2 < n) w[u] |= (uint32_t)q[(e >> 1) + 1] << 8;
                     }
                 }
-                a[u] = __ldg(absmax + (e >> log2B));
+                const int64_t blk = e >> log2B;
+                if constexpr (NESTED)
+                    a[u] = __fadd_rn(__fmul_rn(code_s[NESTED ? 1 : 0][__ldg(ns.qabs + blk)], __ldg(ns.absmax2 + (blk >> 8))),
+                                     off);
+                else
+                    a[u] = __ldg(absmax + blk);
             }
         }
 #pragma unroll
@@ -256,7 +291,7 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
             }
             float y[4];
 #pragma unroll
-            for (int i = 0; i < 4; i++) y[i] = __fmul_rn(cs.code[idx[i]], a[u]);
+            for (int i = 0; i < 4; i++) y[i] = __fmul_rn(code_s[0][idx[i]], a[u]);
             if (e + 4 <= n) {
                 if (BF16OUT) {
                     st_stream_u2(static_cast<uint16_t*>(out) + e,
@@ -293,15 +328,15 @@ bnbq_status persistent_grid(Kern kern, int threads, size_t smem, int64_t work_un
     return BNBQ_OK;
 }
 
-template <int B, bool BF16, int K>
+template <int B, bool BF16, int K, bool CENTER = false>
 bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax, uint8_t* out,
-                     cudaStream_t s)
+                     cudaStream_t s, const float* center = nullptr)
 {
     using Geo = QGeom<B>;
     unsigned* flags = nullptr;
     bnbq_status st = device_flag_ptr(&flags);
     if (st != BNBQ_OK) return st;
-    auto kern = quantize_kernel<B, BF16, K>;
+    auto kern = quantize_kernel<B, BF16, K, CENTER>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -314,7 +349,7 @@ bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax,
     int grid = 0;
     st = persistent_grid(kern, kQThreads, Geo::kSmem, (n + B - 1) / B, Geo::kGroups, &grid);
     if (st != BNBQ_OK) return st;
-    kern<<<grid, kQThreads, Geo::kSmem, s>>>(code, A, n, absmax, out, flags);
+    kern<<<grid, kQThreads, Geo::kSmem, s>>>(code, A, n, absmax, out, flags, center);
     return cuda_status(cudaGetLastError(), "quantize_kernel launch");
 }
 
@@ -334,9 +369,9 @@ bnbq_status launch_q_b(const float* code, int K, const void* A, bnbq_dtype dt, i
                            : launch_q_k<B, false>(code, K, A, n, absmax, out, s);
 }
 
-template <int K, bool BF16OUT>
+template <int K, bool BF16OUT, bool NESTED = false>
 bnbq_status launch_dq(const float* code, const uint8_t* q, const float* absmax, int64_t n, int B,
-                      void* out, cudaStream_t s)
+                      void* out, cudaStream_t s, NestedScales ns = NestedScales{})
 {
     unsigned* flags = nullptr;
     bnbq_status st = device_flag_ptr(&flags);
@@ -344,10 +379,10 @@ bnbq_status launch_dq(const float* code, const uint8_t* q, const float* absmax, 
     int log2B = 0;
     while ((1 << log2B) < B) log2B++;
     int grid = 0;
-    auto kern = dequantize_kernel<K, BF16OUT>;
+    auto kern = dequantize_kernel<K, BF16OUT, NESTED>;
     st = persistent_grid(kern, 256, 0, (n + 3) / 4, 256 * 4, &grid);
     if (st != BNBQ_OK) return st;
-    kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags);
+    kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags, ns);
     return cuda_status(cudaGetLastError(), "dequantize_kernel launch");
 }
 
@@ -357,11 +392,31 @@ bnbq_status launch_quantize(const float* code, int K, const void* A, bnbq_dtype 
                             int B, float* absmax, uint8_t* out, cudaStream_t s)
 {
     switch (B) {
+        case 64: return launch_q_b<64>(code, K, A, dt, n, absmax, out, s);
+        case 128: return launch_q_b<128>(code, K, A, dt, n, absmax, out, s);
         case 256: return launch_q_b<256>(code, K, A, dt, n, absmax, out, s);
         case 2048: return launch_q_b<2048>(code, K, A, dt, n, absmax, out, s);
         case 4096: return launch_q_b<4096>(code, K, A, dt, n, absmax, out, s);
-        default: return fail(BNBQ_EINVAL, "blocksize %d not in {256, 2048, 4096}", B);
+        default: return fail(BNBQ_EINVAL, "blocksize %d not in {64, 128, 256, 2048, 4096}", B);
     }
+}
+
+bnbq_status launch_quantize_centred(const float* code2, const float* a, int64_t nb, const float* center,
+                                    float* absmax2, uint8_t* qabs, cudaStream_t s)
+{
+    return launch_q<kNestBlock, false, 256, true>(code2, a, nb, absmax2, qabs, s, center);
+}
+
+bnbq_status launch_dequantize_nested(const float* code, int K, const uint8_t* q, const uint8_t* qabs,
+                                     const float* absmax2, const float* center, const float* code2, int64_t n,
+                                     int B, void* out, bnbq_dtype dt, cudaStream_t s)
+{
+    const NestedScales ns{qabs, absmax2, center, code2};
+    if (K == 256)
+        return dt == BNBQ_BF16 ? launch_dq<256, true, true>(code, q, nullptr, n, B, out, s, ns)
+                               : launch_dq<256, false, true>(code, q, nullptr, n, B, out, s, ns);
+    return dt == BNBQ_BF16 ? launch_dq<16, true, true>(code, q, nullptr, n, B, out, s, ns)
+                           : launch_dq<16, false, true>(code, q, nullptr, n, B, out, s, ns);
 }
 
 bnbq_status launch_dequantize(const float* code, int K, const uint8_t* q, const float* absmax,

@@ -78,6 +78,7 @@ typedef enum {
  *   code      device, code_size fp32 values, strictly increasing, within [-1, 1]
  *   code_size 256 (8-bit codes, one byte per element) or 16 (two 4-bit codes per byte)
  *   A         device, n elements of a_dtype
+ *   blocksize 64, 128, 256, 2048 or 4096 (64 is the 4-bit weight setting of QLoRA)
  *   absmax    device, out: ceil(n/blocksize) fp32, absmax[b] = max |A_i| over block b
  *   out       device, out: n bytes (code_size 256) or ceil(n/2) bytes (code_size 16; element 2k
  *             in the high nibble of byte k, element 2k+1 in the low nibble; for odd n the last
@@ -99,6 +100,41 @@ BNBQ_API bnbq_status bnbq_quantize_blockwise(const float* code, int code_size, c
 BNBQ_API bnbq_status bnbq_dequantize_blockwise(const float* code, int code_size, const uint8_t* q,
                                       const float* absmax, int64_t n, int blocksize, void* out,
                                       bnbq_dtype out_dtype, bnbq_stream_t stream);
+
+/*
+ * Nested (double) quantization of a block-scale array (page "Bitsandbytes", section "İç içe
+ * nicelleştirme": a second quantization of the quantized weights' constants, about 0.4 bit per
+ * parameter saved; scheme of "QLoRA: Efficient Finetuning of Quantized LLMs", section 3, Double
+ * Quantization).  For absmax[nb] (fp32, >= 0, e.g. from bnbq_quantize_blockwise):
+ *   offset    device, out: 1 fp32, the mean of absmax -- a double sum over chunks of 4096
+ *             consecutive scales (each chunk in index order, then the chunk sums in index
+ *             order), divided by nb in double and rounded once; 0 when nb == 0
+ *   qabs      device, out: nb bytes, absmax2 device, out: ceil(nb/256) fp32 -- the block-wise
+ *             8-bit quantization (blocks of 256, code2) of absmax_i - offset (one fp32
+ *             subtraction), with the rule of bnbq_quantize_blockwise
+ *   code2     device, 256 fp32 (the signed dynamic code is the intended one)
+ *   workspace device, bnbq_nested_workspace_bytes(nb) bytes, 8-byte aligned, caller-owned;
+ *             its contents are scratch.  absmax must be 16-byte aligned.
+ * Asynchronous on `stream`; three kernel launches.
+ */
+BNBQ_API int64_t bnbq_nested_workspace_bytes(int64_t nb);
+BNBQ_API bnbq_status bnbq_quantize_absmax_nested(const float* absmax, int64_t nb, const float* code2,
+                                                 uint8_t* qabs, float* absmax2, float* offset,
+                                                 void* workspace, bnbq_stream_t stream);
+
+/* Rebuild the scales: absmax_out[i] = code2[qabs_i] * absmax2[i/256] + *offset (two fp32
+ * roundings, multiply then add).  All pointers device memory. */
+BNBQ_API bnbq_status bnbq_dequantize_absmax_nested(const uint8_t* qabs, const float* absmax2,
+                                                   const float* offset, const float* code2, int64_t nb,
+                                                   float* absmax_out, bnbq_stream_t stream);
+
+/* bnbq_dequantize_blockwise with each block's scale rebuilt on the fly from its nested
+ * quantization (as bnbq_dequantize_absmax_nested computes it): one pass, no fp32 scale array. */
+BNBQ_API bnbq_status bnbq_dequantize_blockwise_nested(const float* code, int code_size, const uint8_t* q,
+                                                      const uint8_t* qabs, const float* absmax2,
+                                                      const float* offset, const float* code2, int64_t n,
+                                                      int blocksize, void* out, bnbq_dtype out_dtype,
+                                                      bnbq_stream_t stream);
 
 /* One tensor of a multi-tensor optimizer step.  All pointers are device memory. */
 typedef struct {

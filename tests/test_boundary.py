@@ -89,6 +89,29 @@ def test_dequantize_argument_checks():
     assert L.bnbq_dequantize_blockwise(0x1000, 256, None, None, 0, 256, None, 0, None) == B.OK
 
 
+def test_nested_argument_checks():
+    """Nested quantization of block scales: checks before any CUDA call."""
+    L = B.lib()
+    assert L.bnbq_nested_workspace_bytes(0) == 0
+    assert L.bnbq_nested_workspace_bytes(1) == 8
+    assert L.bnbq_nested_workspace_bytes(4096) == 8 and L.bnbq_nested_workspace_bytes(4097) == 16
+    q = L.bnbq_quantize_absmax_nested
+    assert q(0x1000, -1, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == B.EINVAL
+    assert q(0x1000, 10, None, 0x3000, 0x4000, 0x5000, 0x6000, None) == B.EINVAL        # no code2
+    assert q(0x1000, 10, 0x2000, 0x3000, 0x4000, 0x5000, None, None) == B.EINVAL        # no workspace
+    assert q(0x1004, 10, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == B.EINVAL      # absmax alignment
+    assert q(0x1000, 10, 0x2000, 0x3000, 0x4000, 0x5000, 0x6004, None) == B.EINVAL      # workspace alignment
+    assert "aligned" in B.bnbq_last_error()
+    d = L.bnbq_dequantize_absmax_nested
+    assert d(0x1000, 0x2000, 0x3000, 0x4000, -1, 0x5000, None) == B.EINVAL
+    assert d(None, None, None, None, 0, None, None) == B.OK                               # empty: no-op
+    dn = L.bnbq_dequantize_blockwise_nested
+    assert dn(0x1000, 16, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 100, 32, 0x7000, 0, None) == B.EINVAL  # blocksize
+    assert dn(0x1000, 16, 0x2000, 0x3000, 0x4000, 0x5000, None, 100, 64, 0x7000, 0, None) == B.EINVAL    # no code2
+    assert dn(0x1000, 16, 0x2001, 0x3000, 0x4000, 0x5000, 0x6000, 100, 64, 0x7000, 0, None) == B.EINVAL  # q alignment
+    assert dn(0x1000, 16, None, None, None, None, 0x6000, 0, 64, None, 0, None) == B.OK
+
+
 def _t(**kw):
     d = dict(p=0x10000, g=0x20000, state1=0x30000, state2=0x40000, absmax1=0x50000, absmax2=0x60000, n=5000,
              g_dtype=1, state_bits=8)

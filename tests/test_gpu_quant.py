@@ -1,7 +1,8 @@
 """GPU parity: block-wise quantize / dequantize through the C ABI against the CPU oracle.
 
 Workload: the standalone quantize + dequantize sweep -- fp32 and bf16 tensors, N(0,1) with 0.1%
-of positions scaled x50, blocksize 256/2048/4096, 8-bit signed dynamic code and NF4 (seed 1).
+of positions scaled x50, blocksize 256/2048/4096 (and 64/128, the 4-bit weight setting), 8-bit
+signed dynamic code and NF4 (seed 1).
 2^20-element tensors (plus a ragged tail) are compared element by element; the 2^24 and 2^28
 tensors are run whole, in the launch configuration of the benchmark, and compared on sampled
 blocks that the oracle recomputes one by one (blocks are independent).  Bar: bit-exact codes,
@@ -87,7 +88,7 @@ def _check_full(code_cpu, x, B):
 
 
 @pytest.mark.parametrize("code_name", ["signed", "nf4"])
-@pytest.mark.parametrize("B", [256, 2048, 4096])
+@pytest.mark.parametrize("B", [64, 128, 256, 2048, 4096])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_sweep_2p20_elementwise(code_name, B, dtype):
     code = _codes()[code_name]
