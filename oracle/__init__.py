@@ -55,7 +55,7 @@ def lib():
             L = ctypes.CDLL(_LIB)
             vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             for name in ("oracle_code_dynamic_unsigned", "oracle_code_dynamic_signed",
-                         "oracle_code_nf4", "oracle_code_linear"):
+                         "oracle_code_nf4", "oracle_code_fp4", "oracle_code_linear"):
                 getattr(L, name).argtypes = [vp]
                 getattr(L, name).restype = None
             L.oracle_code_mid.argtypes = [vp, i32]
@@ -105,6 +105,12 @@ def code_dynamic_signed() -> np.ndarray:
 def code_nf4() -> np.ndarray:
     out = np.zeros(16, np.float32)
     lib().oracle_code_nf4(_ptr(out))
+    return out
+
+
+def code_fp4() -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    lib().oracle_code_fp4(_ptr(out))
     return out
 
 

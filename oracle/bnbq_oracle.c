@@ -117,6 +117,30 @@ void oracle_code_nf4(float out[16])
     sort_floats(out, 16);
 }
 
+/* FP4 [FP4]: the 4-bit float E2M1 -- a sign bit, 2 exponent bits (bias 1) and 1 mantissa bit,
+ * subnormals and no inf/NaN, so the magnitudes are 0, 0.5 (subnormal) and 2^(e-1) * (1 + f/2)
+ * for e = 1..3, f = 0..1: 1, 1.5, 2, 3, 4, 6 -- divided by the largest, 6, so -1, 0 and +1 are
+ * exact.  READING: E2M1 has two zeros; the codebook must be strictly increasing, so the -0
+ * pattern is given the next finer subnormal magnitude, 0.25/6 (as the signed dynamic code gives
+ * its -0 pattern the next tree level).  16 values, formed in double and rounded once. */
+void oracle_code_fp4(float out[16])
+{
+    int c = 0;
+    for (int sign = -1; sign <= 1; sign += 2) {
+        for (int e = 0; e <= 3; e++) {
+            for (int f = 0; f <= 1; f++) {
+                double mag = (e == 0) ? 0.5 * (double)f : ldexp(1.0 + 0.5 * (double)f, e - 1);
+                if (sign < 0 && e == 0 && f == 0) {
+                    out[c++] = (float)(0.25 / 6.0); /* the -0 pattern */
+                    continue;
+                }
+                out[c++] = (float)((double)sign * mag / 6.0);
+            }
+        }
+    }
+    sort_floats(out, 16);
+}
+
 /* Linear (uniform) code over [-1, 1], used by tests only. */
 void oracle_code_linear(float out[256])
 {

@@ -31,6 +31,9 @@
  *  [QLORA] T. Dettmers et al., "QLoRA: Efficient Finetuning of Quantized LLMs", section 3
  *          (NormalFloat: quantiles of N(0,1), asymmetric 8+7 split with one shared zero;
  *          Double Quantization: the constants quantized again, 8-bit, blocks of 256, centred).
+ *  [FP4]   page "Quantize 🤗 Transformers models", section "FP4 quantization" (4-bit loading with
+ *          the FP4 data type); the format is the E2M1 4-bit float of the OCP Microscaling
+ *          Formats (MX) specification v1.0, section 5.3.3.
  *  [NEST]  page "Bitsandbytes" (transformers docs, Turkish), section "İç içe nicelleştirme"
  *          (nested quantization: a second quantization of the already quantized weights'
  *          constants, about 0.4 bit per parameter saved).
@@ -66,6 +69,7 @@ typedef struct {
 void oracle_code_dynamic_unsigned(float out[256]);
 void oracle_code_dynamic_signed(float out[256]);
 void oracle_code_nf4(float out[16]);
+void oracle_code_fp4(float out[16]);
 void oracle_code_linear(float out[256]);
 
 /* mid_j of the nearest-code rule, j = 0..K-2 */

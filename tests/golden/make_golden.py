@@ -28,6 +28,11 @@ SOURCES = {
         "construction from Dettmers et al., 'QLoRA', section 3.\n"
         "reading: N(0,1) quantiles at probabilities delta + (1/2-delta) k/7 (k=0..6), zero, and "
         "1/2 + (1/2-delta) k/8 (k=1..8), divided by the largest; delta = (1/30 + 1/32)/2.  16 values."),
+    "code_fp4": (
+        "source: FP4 data type, page 'Quantize 🤗 Transformers models', section 'FP4 quantization'; "
+        "format E2M1 of the OCP Microscaling Formats (MX) specification v1.0, section 5.3.3.\n"
+        "reading: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 with both signs, divided by 6; the negative-zero "
+        "pattern takes 0.25/6 so the table is strictly increasing.  16 values, ascending."),
     "code_linear": (
         "source: 'linear quantization' in the feature list of the page "
         "'Py之bitsandbytes：bitsandbytes的简介、安装、使用方法之详细攻略', section 1.\n"

@@ -112,6 +112,19 @@ def test_nf4_normal_quantiles(oracle_mod):
     np.testing.assert_array_equal(c.astype(np.float32), want.astype(np.float32))
 
 
+def test_fp4_e2m1_values(oracle_mod):
+    """FP4 = E2M1 (page "Quantize 🤗 Transformers models", section "FP4 quantization"; OCP MX v1.0):
+    written out by hand, the sixteen values are k/12 for k in {0, 1, 2, 3, 4, 6, 8, 12} with both
+    signs, the spare negative zero replaced by 1/24, each rounded once to binary32."""
+    c = oracle_mod.code_fp4()
+    want = sorted({Fraction(s * k, 12) for s in (-1, 1) for k in (0, 1, 2, 3, 4, 6, 8, 12)} | {Fraction(1, 24)})
+    assert len(want) == 16
+    np.testing.assert_array_equal(c, np.array([float(w) for w in want]).astype(np.float32))
+    assert c[0] == -1.0 and c[-1] == 1.0 and 0.0 in c
+    # away from zero the table is symmetric: E2M1 has the same magnitudes for both signs
+    np.testing.assert_array_equal(-c[:7][::-1], c[9:])
+
+
 def test_linear_code(oracle_mod):
     c = oracle_mod.code_linear()
     assert c[0] == -1.0 and c[-1] == 1.0
@@ -120,7 +133,8 @@ def test_linear_code(oracle_mod):
 
 def test_midpoints_exact_for_dynamic_codes(oracle_mod):
     """mid_j is the exact mean of neighbours whenever that mean is a binary32 number."""
-    for code in (oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned(), oracle_mod.code_nf4()):
+    for code in (oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned(), oracle_mod.code_nf4(),
+                 oracle_mod.code_fp4()):
         for j in range(len(code) - 1):
             exact = (Fraction(float(code[j])) + Fraction(float(code[j + 1]))) / 2
             mid = oracle_mod.code_mid(code, j)
@@ -140,7 +154,8 @@ def _read_hex(path):
 
 @pytest.mark.parametrize("name,fn", [("code_dynamic_signed", "code_dynamic_signed"),
                                      ("code_dynamic_unsigned", "code_dynamic_unsigned"),
-                                     ("code_nf4", "code_nf4"), ("code_linear", "code_linear")])
+                                     ("code_nf4", "code_nf4"), ("code_fp4", "code_fp4"),
+                                     ("code_linear", "code_linear")])
 def test_golden_codebooks(oracle_mod, name, fn):
     path = os.path.join(GOLDEN, name + ".hex")
     with open(path) as f:
