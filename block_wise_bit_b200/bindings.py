@@ -20,9 +20,9 @@ OK, EINVAL, EUNSUPPORTED, ECUDA = 0, 1, 2, 3
 F32, BF16 = 0, 1
 ADAMW, ADAM, LION, MOMENTUM, RMSPROP = 0, 1, 2, 3, 4
 OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM, "rmsprop": RMSPROP}
-CODE_DYNAMIC_SIGNED, CODE_DYNAMIC_UNSIGNED, CODE_NF4, CODE_LINEAR = 0, 1, 2, 3
+CODE_DYNAMIC_SIGNED, CODE_DYNAMIC_UNSIGNED, CODE_NF4, CODE_LINEAR, CODE_FP4 = 0, 1, 2, 3, 4
 CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DYNAMIC_UNSIGNED,
-              "nf4": CODE_NF4, "linear": CODE_LINEAR}
+              "nf4": CODE_NF4, "linear": CODE_LINEAR, "fp4": CODE_FP4}
 FLAG_BAD_CODE, FLAG_NONFINITE = 0x1, 0x2
 
 EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_step_8bit_noalloc",

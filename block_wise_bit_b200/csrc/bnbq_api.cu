@@ -282,6 +282,28 @@ void build_nf4(float* out)
     for (int k = 1; k <= 8; k++) out[c++] = (float)(std_normal_quantile(0.5 + (0.5 - delta) * k / 8.0) / top);
 }
 
+// FP4: the E2M1 4-bit float (page "Quantize 🤗 Transformers models", section "FP4 quantization";
+// OCP Microscaling Formats v1.0, section 5.3.3) decoded from its 16 bit patterns -- sign, two
+// exponent bits with bias 1, one mantissa bit, subnormals at exponent 0 -- divided by the largest
+// magnitude 6 and sorted.  The negative-zero pattern, a duplicate of zero, takes the next finer
+// subnormal step 0.25 so that the table is strictly increasing.
+void build_fp4(float* out)
+{
+    double v[16];
+    for (int b = 0; b < 16; b++) {
+        const int sgn = b >> 3, e = (b >> 1) & 3, m = b & 1;
+        const double mag = e == 0 ? 0.5 * m : (1.0 + 0.5 * m) * (double)(1 << (e - 1));
+        v[b] = (b == 8) ? 0.25 / 6.0 : (sgn ? -mag : mag) / 6.0;
+    }
+    for (int i = 1; i < 16; i++)
+        for (int j = i; j > 0 && v[j - 1] > v[j]; j--) {
+            const double t = v[j];
+            v[j] = v[j - 1];
+            v[j - 1] = t;
+        }
+    for (int i = 0; i < 16; i++) out[i] = (float)v[i];
+}
+
 void build_linear(float* out)
 {
     for (int k = 0; k < 256; k++) out[k] = (float)(-1.0 + 2.0 * k / 255.0);
@@ -307,7 +329,8 @@ int bnbq_code_size(bnbq_code_kind kind)
         case BNBQ_CODE_DYNAMIC_SIGNED:
         case BNBQ_CODE_DYNAMIC_UNSIGNED:
         case BNBQ_CODE_LINEAR: return 256;
-        case BNBQ_CODE_NF4: return 16;
+        case BNBQ_CODE_NF4:
+        case BNBQ_CODE_FP4: return 16;
         default: return -1;
     }
 }
@@ -319,6 +342,7 @@ int bnbq_codebook(bnbq_code_kind kind, float* out)
         case BNBQ_CODE_DYNAMIC_SIGNED: build_dynamic(true, out); return 256;
         case BNBQ_CODE_DYNAMIC_UNSIGNED: build_dynamic(false, out); return 256;
         case BNBQ_CODE_NF4: build_nf4(out); return 16;
+        case BNBQ_CODE_FP4: build_fp4(out); return 16;
         case BNBQ_CODE_LINEAR: build_linear(out); return 256;
         default: return -1;
     }

@@ -65,7 +65,8 @@ typedef enum {
     BNBQ_CODE_DYNAMIC_SIGNED = 0,   /* 256 values, for m / Lion / momentum state */
     BNBQ_CODE_DYNAMIC_UNSIGNED = 1, /* 256 values, for Adam's v */
     BNBQ_CODE_NF4 = 2,              /* 16 values */
-    BNBQ_CODE_LINEAR = 3            /* 256 values, -1 + 2k/255 */
+    BNBQ_CODE_LINEAR = 3,           /* 256 values, -1 + 2k/255 */
+    BNBQ_CODE_FP4 = 4               /* 16 values: E2M1 4-bit float / 6, the -0 pattern as +0.25/6 */
 } bnbq_code_kind;
 
 /* device flag bits (bnbq_device_flags) */

@@ -41,7 +41,7 @@ def test_only_bnbq_symbols_exported():
     assert funcs and all(f.startswith("bnbq_") for f in funcs), funcs
 
 
-@pytest.mark.parametrize("kind", ["dynamic_signed", "dynamic_unsigned", "nf4", "linear"])
+@pytest.mark.parametrize("kind", ["dynamic_signed", "dynamic_unsigned", "nf4", "fp4", "linear"])
 def test_library_codebooks_match_oracle_and_golden(oracle_mod, kind):
     lib_code = B.bnbq_codebook(kind).numpy()
     np.testing.assert_array_equal(lib_code, getattr(oracle_mod, "code_" + kind)())

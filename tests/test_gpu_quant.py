@@ -33,7 +33,7 @@ def _cuda():
 
 
 def _codes():
-    return {"signed": bq.bnbq_codebook("dynamic_signed"), "nf4": bq.bnbq_codebook("nf4"),
+    return {"signed": bq.bnbq_codebook("dynamic_signed"), "nf4": bq.bnbq_codebook("nf4"), "fp4": bq.bnbq_codebook("fp4"),
             "unsigned": bq.bnbq_codebook("dynamic_unsigned"), "linear": bq.bnbq_codebook("linear")}
 
 
@@ -87,7 +87,7 @@ def _check_full(code_cpu, x, B):
     return a, q
 
 
-@pytest.mark.parametrize("code_name", ["signed", "nf4"])
+@pytest.mark.parametrize("code_name", ["signed", "nf4", "fp4"])
 @pytest.mark.parametrize("B", [64, 128, 256, 2048, 4096])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_sweep_2p20_elementwise(code_name, B, dtype):
