@@ -53,13 +53,18 @@ WORKLOADS = {
 }
 
 # Standalone quantize / dequantize sweep points (development measurements of those kernels):
-# name: (log2 n, input dtype, codebook, blocksize)
+# name: (log2 n, input dtype, codebook, blocksize, nested block scales)
 QUANT_WORKLOADS = {
-    "quant_2p28_f32_signed_b2048": (28, "f32", "dynamic_signed", 2048),
-    "quant_2p28_bf16_signed_b2048": (28, "bf16", "dynamic_signed", 2048),
-    "quant_2p28_f32_nf4_b2048": (28, "f32", "nf4", 2048),
-    "quant_2p28_f32_signed_b256": (28, "f32", "dynamic_signed", 256),
-    "quant_2p28_f32_signed_b4096": (28, "f32", "dynamic_signed", 4096),
+    "quant_2p28_f32_signed_b2048": (28, "f32", "dynamic_signed", 2048, False),
+    "quant_2p28_bf16_signed_b2048": (28, "bf16", "dynamic_signed", 2048, False),
+    "quant_2p28_f32_nf4_b2048": (28, "f32", "nf4", 2048, False),
+    "quant_2p28_f32_signed_b256": (28, "f32", "dynamic_signed", 256, False),
+    "quant_2p28_f32_signed_b4096": (28, "f32", "dynamic_signed", 4096, False),
+    # 4-bit weights as QLoRA stores them: blocksize 64, NF4 or FP4, bf16 weights
+    "quant_2p28_bf16_nf4_b64": (28, "bf16", "nf4", 64, False),
+    "quant_2p28_bf16_fp4_b64": (28, "bf16", "fp4", 64, False),
+    # ... with the block scales nested (quantize + nest; dequantize rebuilding the scales)
+    "quant_2p28_bf16_nf4_b64_nested": (28, "bf16", "nf4", 64, True),
 }
 
 
@@ -69,7 +74,7 @@ def bench_quant(args, base):
     import torch
     import block_wise_bit_b200 as bq
     from block_wise_bit_b200 import workloads as W
-    log2n, dt, code_name, B = QUANT_WORKLOADS[args.workload]
+    log2n, dt, code_name, B, nested = QUANT_WORKLOADS[args.workload]
     n = 1 << log2n
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
@@ -84,19 +89,35 @@ def bench_quant(args, base):
     y = torch.empty(n, dtype=dtype, device=dev)
     esz = x.element_size()
     qbytes = n if K == 256 else n / 2
-    alg_q = n * esz + qbytes + 4 * absmax.numel()
-    alg_dq = qbytes + 4 * absmax.numel() + n * esz
+    nb = absmax.numel()
+    alg_q = n * esz + qbytes + 4 * nb
+    alg_dq = qbytes + 4 * nb + n * esz
     stream = torch.cuda.current_stream(dev)
-    for _ in range(args.warmup):
+    if nested:  # nest: read the scales twice (mean, quantize), write codes + second-level scales
+        code2 = bq.bnbq_codebook("dynamic_signed").to(dev)
+        nb2 = (nb + 255) // 256
+        alg_q += 8 * nb + nb + 4 * nb2
+        alg_dq = qbytes + nb + 4 * nb2 + n * esz
+
+    def quantize():
         bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
-        bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
+        return bq.bnbq_quantize_absmax_nested(code2, absmax) if nested else None
+
+    def dequantize(nest):
+        if nested:
+            bq.bnbq_dequantize_blockwise_nested(code, q, *nest, code2, n, B, out=y)
+        else:
+            bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
+
+    for _ in range(args.warmup):
+        dequantize(quantize())
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     for k in range(args.steps):
         evs[k][0].record(stream)
-        bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
+        nest = quantize()
         evs[k][1].record(stream)
-        bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
+        dequantize(nest)
         evs[k][2].record(stream)
     torch.cuda.synchronize()
     tq = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
@@ -105,10 +126,11 @@ def bench_quant(args, base):
     out = dict(base, metric="block-wise quantize + dequantize elements/s", unit="elements/s",
                value=n / ((tq + td) / 1e3), n_gpus=1, steps=args.steps, warmup=args.warmup,
                ms_per_step=round(tq + td, 4), dtype=dt,
-               config={"workload": args.workload, "n": n, "blocksize": B, "codebook": code_name},
+               config={"workload": args.workload, "n": n, "blocksize": B, "codebook": code_name,
+                       "nested_scales": nested},
                quantize={"ms": round(tq, 4), "GB/s": round(alg_q / tq / 1e6, 1), "frac": round(alg_q / tq / 1e6 / peak, 4)},
                dequantize={"ms": round(td, 4), "GB/s": round(alg_dq / td / 1e6, 1), "frac": round(alg_dq / td / 1e6 / peak, 4)},
-               peak_gbs=peak, gpu_launches=2 * args.steps)
+               peak_gbs=peak, gpu_launches=(5 if nested else 2) * args.steps)
     print(json.dumps(out))
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
