@@ -32,7 +32,7 @@
 #define BNBQ_STEP_EPT 16
 #endif
 #ifndef BNBQ_STEP_THREADS
-#define BNBQ_STEP_THREADS 768        // CTA size for blocksize 256 and 4096
+#define BNBQ_STEP_THREADS 1024       // CTA size for blocksize 256 and 4096
 #endif
 #ifndef BNBQ_STEP_THREADS_2048
 #define BNBQ_STEP_THREADS_2048 BNBQ_STEP_THREADS  // CTA size for blocksize 2048
