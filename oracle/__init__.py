@@ -47,36 +47,56 @@ class _HP(ctypes.Structure):
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
 
 
+def _declare(L):
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    for name in ("oracle_code_dynamic_unsigned", "oracle_code_dynamic_signed",
+                 "oracle_code_nf4", "oracle_code_fp4", "oracle_code_linear"):
+        getattr(L, name).argtypes = [vp]
+        getattr(L, name).restype = None
+    L.oracle_code_mid.argtypes = [vp, i32]
+    L.oracle_code_mid.restype = ctypes.c_float
+    L.oracle_nearest_code.argtypes = [vp, i32, ctypes.c_float]
+    L.oracle_nearest_code.restype = i32
+    L.oracle_quantize_blockwise.argtypes = [vp, i32, vp, i32, i64, i32, vp, vp]
+    L.oracle_quantize_blockwise.restype = i32
+    L.oracle_dequantize_blockwise.argtypes = [vp, i32, vp, vp, i64, i32, vp, i32]
+    L.oracle_dequantize_blockwise.restype = i32
+    L.oracle_step_blocks.argtypes = [i32, i32, vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, i32,
+                                     ctypes.POINTER(_HP), i32, i64, i64]
+    L.oracle_step_blocks.restype = i32
+    L.oracle_absmax_mean.argtypes = [vp, i64]
+    L.oracle_absmax_mean.restype = ctypes.c_float
+    L.oracle_nest_absmax.argtypes = [vp, i64, vp, vp, vp, vp]
+    L.oracle_nest_absmax.restype = i32
+    L.oracle_unnest_absmax.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp]
+    L.oracle_unnest_absmax.restype = i32
+    return L
+
+
 def lib():
     global _lib
     with _lock:
         if _lib is None:
             build()
-            L = ctypes.CDLL(_LIB)
-            vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-            for name in ("oracle_code_dynamic_unsigned", "oracle_code_dynamic_signed",
-                         "oracle_code_nf4", "oracle_code_fp4", "oracle_code_linear"):
-                getattr(L, name).argtypes = [vp]
-                getattr(L, name).restype = None
-            L.oracle_code_mid.argtypes = [vp, i32]
-            L.oracle_code_mid.restype = ctypes.c_float
-            L.oracle_nearest_code.argtypes = [vp, i32, ctypes.c_float]
-            L.oracle_nearest_code.restype = i32
-            L.oracle_quantize_blockwise.argtypes = [vp, i32, vp, i32, i64, i32, vp, vp]
-            L.oracle_quantize_blockwise.restype = i32
-            L.oracle_dequantize_blockwise.argtypes = [vp, i32, vp, vp, i64, i32, vp, i32]
-            L.oracle_dequantize_blockwise.restype = i32
-            L.oracle_step_blocks.argtypes = [i32, i32, vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, i32,
-                                             ctypes.POINTER(_HP), i32, i64, i64]
-            L.oracle_step_blocks.restype = i32
-            L.oracle_absmax_mean.argtypes = [vp, i64]
-            L.oracle_absmax_mean.restype = ctypes.c_float
-            L.oracle_nest_absmax.argtypes = [vp, i64, vp, vp, vp, vp]
-            L.oracle_nest_absmax.restype = i32
-            L.oracle_unnest_absmax.argtypes = [vp, vp, ctypes.c_float, vp, i64, vp]
-            L.oracle_unnest_absmax.restype = i32
-            _lib = L
+            _lib = _declare(ctypes.CDLL(_LIB))
     return _lib
+
+
+def swap_library(path):
+    """Test hook: load another build of this oracle's source (the mutation tests plant a mistake
+    in a copy of it) in place of the real one; returns the previous library handle, which
+    ``restore_library`` puts back."""
+    global _lib
+    with _lock:
+        prev = _lib
+        _lib = _declare(ctypes.CDLL(path))
+    return prev
+
+
+def restore_library(prev):
+    global _lib
+    with _lock:
+        _lib = prev
 
 
 def _ptr(a):
