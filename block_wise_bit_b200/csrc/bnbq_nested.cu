@@ -9,26 +9,29 @@
 // 8/64 + 32/(64*256) bits per weight for the scales instead of 32/64.
 //
 // The mean is a plain double sum in a fixed order -- chunks of kNestChunk consecutive scales,
-// each summed in index order by one thread, then the chunk sums in index order by one thread --
+// each summed in index order (one CTA per chunk), then the chunk sums in index order --
 // divided by nb in double and rounded once to binary32, so every run (and the CPU restatement)
-// gets the same offset.  This is a one-off pass over nb = n/64 scales, far off the step's path;
-// it is kept simple rather than fast.
+// gets the same offset.  This is a one-off pass over nb = n/64 scales, far off the step's path.
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 
 namespace bnbq {
 namespace {
 
+// One CTA per chunk: the chunk is staged in shared memory with coalesced loads, then one
+// thread adds it up in index order (the order is part of the definition of the offset).
 __global__ void __launch_bounds__(256)
 absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ work)
 {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t start = c * kNestChunk;
-    if (start >= nb) return;
-    const int64_t end = (start + kNestChunk < nb) ? start + kNestChunk : nb;
+    __shared__ float chunk[kNestChunk];
+    const int64_t start = (int64_t)blockIdx.x * kNestChunk;
+    const int len = (int)((nb - start < kNestChunk) ? nb - start : kNestChunk);
+    for (int i = threadIdx.x; i < len; i += blockDim.x) chunk[i] = __ldg(a + start + i);
+    __syncthreads();
+    if (threadIdx.x != 0) return;
     double s = 0.0;
-    for (int64_t i = start; i < end; i++) s = __dadd_rn(s, (double)__ldg(a + i));
-    work[c] = s;
+    for (int i = 0; i < len; i++) s = __dadd_rn(s, (double)chunk[i]);
+    work[blockIdx.x] = s;
 }
 
 __global__ void __launch_bounds__(32)
@@ -68,7 +71,7 @@ bool aligned_n(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>
 bnbq_status launch_absmax_mean(const float* a, int64_t nb, double* work, float* center, cudaStream_t s)
 {
     const int64_t nchunks = (nb + kNestChunk - 1) / kNestChunk;
-    absmax_chunk_sums<<<(unsigned)((nchunks + 255) / 256), 256, 0, s>>>(a, nb, work);
+    absmax_chunk_sums<<<(unsigned)nchunks, 256, 0, s>>>(a, nb, work);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "absmax_chunk_sums launch");
     absmax_mean_finish<<<1, 32, 0, s>>>(work, nchunks, nb, center);

@@ -207,7 +207,12 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
         quantize_loop<B, BF16, K, kSearchSigned, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
 }
 
-// Dequantize: flat grid over 4-element chunks; each thread takes 4 chunks per pass.
+// Dequantize: a lane's unit is 16 bytes of output (8 bf16 or 4 fp32 elements, always inside one
+// block); consecutive lanes take consecutive units, so every load and store instruction of a warp
+// covers one contiguous range.  8-bit codes: one
+// table lookup per element, one packed product per pair.  4-bit codes: a 256-entry table of code
+// pairs indexed by the whole byte (high nibble = the even element): one shared load and one
+// packed product per two elements.
 // NESTED: the block scales are rebuilt from their nested quantization,
 // A_b = code2[qabs_b] * absmax2[b / 256] + *center (two roundings), instead of read from absmax.
 struct NestedScales {
@@ -217,95 +222,130 @@ struct NestedScales {
     const float* code2;
 };
 
+constexpr int kDqUnits = 4;  // units per lane per span
+
+template <bool BF16OUT>
+struct DqGeom {
+    static constexpr int kUnit = BF16OUT ? 8 : 4;      // elements per unit
+    static constexpr int kSpan = 32 * kDqUnits * kUnit;
+};
+
+template <int K, int E>
+struct DqWords {  // the unit's code bytes
+    static constexpr int kBytes = K == 256 ? E : E / 2;
+    static constexpr int kWords = (kBytes + 3) / 4;
+};
+
 template <int K, bool BF16OUT, bool NESTED>
 __global__ void __launch_bounds__(256)
 dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
                   const float* __restrict__ absmax, int64_t n, int log2B, void* __restrict__ out,
-                  unsigned* flags, NestedScales ns)
+                  unsigned* flags, NestedScales ns, bool out16)
 {
+    using Geo = DqGeom<BF16OUT>;
+    constexpr int UE = Geo::kUnit;
+    using Wd = DqWords<K, UE>;
     __shared__ float code_s[NESTED ? 2 : 1][256];
     __shared__ float mid_s[NESTED ? 2 : 1][256];
+    __shared__ float2 pair_s[K == 16 ? 256 : 1];  // 4-bit: byte -> (code[hi nibble], code[lo nibble])
     stage_codes(code_s[0], code, K);
     if constexpr (NESTED) stage_codes(code_s[NESTED ? 1 : 0], ns.code2, 256);
     __syncthreads();
     bool bad = false, tiny = false;
     stage_midpoints(code_s[0], mid_s[0], K, bad, tiny);
     if constexpr (NESTED) stage_midpoints(code_s[NESTED ? 1 : 0], mid_s[NESTED ? 1 : 0], 256, bad, tiny);
+    if constexpr (K == 16)
+        for (int b = threadIdx.x; b < 256; b += blockDim.x) pair_s[b] = make_float2(code_s[0][b >> 4], code_s[0][b & 15]);
     if (__syncthreads_or(bad)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
         return;
     }
     const float off = NESTED ? __ldg(ns.center) : 0.0f;
-
-    const int64_t nchunks = (n + 3) / 4;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < nchunks; c0 += 4 * stride) {
-        uint32_t w[4];
-        float a[4];
+    // Unit j of a pass: fp32 output -- grid-stride units (a thread's units lie far apart);
+    // bf16 output -- warp spans (a warp's units are one contiguous range).  Measured faster each.
+    const int lane = threadIdx.x & 31;
+    const int64_t nspans = (n + Geo::kSpan - 1) / Geo::kSpan;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t threads = (int64_t)gridDim.x * blockDim.x;
+    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    auto unit_start = [&](int64_t span, int j) -> int64_t {
+        if constexpr (BF16OUT) return span * Geo::kSpan + (int64_t)UE * (32 * j + lane);
+        else return (int64_t)UE * (span * (kDqUnits * threads) + j * threads + gtid);
+    };
+    const int64_t first = BF16OUT ? (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5) : 0;
+    const int64_t step = BF16OUT ? warps : 1;
+    const int64_t npass = BF16OUT ? nspans : ((n + UE - 1) / UE + kDqUnits * threads - 1) / (kDqUnits * threads);
+    for (int64_t span = first; span < npass; span += step) {
+        uint32_t w[kDqUnits][Wd::kWords];
+        float a[kDqUnits];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int64_t c = c0 + u * stride;
-            w[u] = 0;
-            a[u] = 0.0f;
-            if (c < nchunks) {
-                const int64_t e = 4 * c;
-                if (K == 256) {
-                    if (e + 4 <= n) {
-                        w[u] = ld_stream_u32(q + e);
+        for (int j = 0; j < kDqUnits; j++) {
+            const int64_t e = unit_start(span, j);
+#pragma unroll
+            for (int t = 0; t < Wd::kWords; t++) w[j][t] = 0;
+            a[j] = 0.0f;
+            if (e < n) {
+                const uint8_t* qb = q + (K == 256 ? e : (e >> 1));
+                if (e + UE <= n) {
+                    if constexpr (Wd::kBytes == 2) {
+                        w[j][0] = (uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(qb));
+                    } else if constexpr (Wd::kBytes == 4 && K == 16) {  // 2-byte aligned codes
+                        w[j][0] = (uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(qb)) |
+                                  ((uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(qb + 2)) << 16);
                     } else {
-                        for (int i = 0; i < 4; i++)
-                            if (e + i < n) w[u] |= (uint32_t)q[e + i] << (8 * i);
+#pragma unroll
+                        for (int t = 0; t < Wd::kWords; t++) w[j][t] = ld_stream_u32(qb + 4 * t);
                     }
-                } else {
-                    if (e + 4 <= n) {
-                        w[u] = __ldcs(reinterpret_cast<const unsigned short*>(q + (e >> 1)));
-                    } else {
-                        w[u] = q[e >> 1];
-                        if (e + 2 < n) w[u] |= (uint32_t)q[(e >> 1) + 1] << 8;
-                    }
+                } else {  // last, partial unit: bytes past the end read as code 0 and are not stored
+                    const int nbytes = (int)(K == 256 ? n - e : (n - e + 1) / 2);
+                    for (int i = 0; i < nbytes; i++) w[j][i >> 2] |= (uint32_t)qb[i] << (8 * (i & 3));
                 }
                 const int64_t blk = e >> log2B;
                 if constexpr (NESTED)
-                    a[u] = __fadd_rn(__fmul_rn(code_s[NESTED ? 1 : 0][__ldg(ns.qabs + blk)], __ldg(ns.absmax2 + (blk >> 8))),
-                                     off);
+                    a[j] = __fadd_rn(__fmul_rn(code_s[NESTED ? 1 : 0][__ldg(ns.qabs + blk)],
+                                               __ldg(ns.absmax2 + (blk >> 8))), off);
                 else
-                    a[u] = __ldg(absmax + blk);
+                    a[j] = __ldg(absmax + blk);
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int64_t c = c0 + u * stride;
-            if (c >= nchunks) continue;
-            const int64_t e = 4 * c;
-            uint32_t idx[4];
-            if (K == 256) {
-                idx[0] = w[u] & 0xff;
-                idx[1] = (w[u] >> 8) & 0xff;
-                idx[2] = (w[u] >> 16) & 0xff;
-                idx[3] = w[u] >> 24;
-            } else {
-                idx[0] = (w[u] >> 4) & 0xf;
-                idx[1] = w[u] & 0xf;
-                idx[2] = (w[u] >> 12) & 0xf;
-                idx[3] = (w[u] >> 8) & 0xf;
-            }
-            float y[4];
+        for (int j = 0; j < kDqUnits; j++) {
+            const int64_t e = unit_start(span, j);
+            if (e >= n) continue;
+            const float2 ap = make_float2(a[j], a[j]);
+            float2 y[UE / 2];
 #pragma unroll
-            for (int i = 0; i < 4; i++) y[i] = __fmul_rn(code_s[0][idx[i]], a[u]);
-            if (e + 4 <= n) {
-                if (BF16OUT) {
-                    st_stream_u2(static_cast<uint16_t*>(out) + e,
-                                 make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3])));
+            for (int h = 0; h < UE / 2; h++) {
+                if constexpr (K == 256) {
+                    const uint32_t wd = w[j][h >> 1];
+                    const uint32_t b0 = 2u * (h & 1);
+                    y[h] = mul2(make_float2(code_s[0][__byte_perm(wd, 0u, 0x4440u + b0)],
+                                            code_s[0][__byte_perm(wd, 0u, 0x4441u + b0)]), ap);
                 } else {
-                    st_stream_f4(static_cast<float*>(out) + e, make_float4(y[0], y[1], y[2], y[3]));
+                    y[h] = mul2(pair_s[__byte_perm(w[j][0], 0u, 0x4440u + h)], ap);
+                }
+            }
+            if (e + UE <= n) {
+                if constexpr (BF16OUT) {
+                    const uint4 v = make_uint4(pack_bf16x2(y[0].x, y[0].y), pack_bf16x2(y[1].x, y[1].y),
+                                               pack_bf16x2(y[2].x, y[2].y), pack_bf16x2(y[3].x, y[3].y));
+                    uint16_t* o = static_cast<uint16_t*>(out) + e;
+                    if (out16) {
+                        __stcs(reinterpret_cast<uint4*>(o), v);
+                    } else {
+                        st_stream_u2(o, make_uint2(v.x, v.y));
+                        st_stream_u2(o + 4, make_uint2(v.z, v.w));
+                    }
+                } else {
+                    st_stream_f4(static_cast<float*>(out) + e, make_float4(y[0].x, y[0].y, y[1].x, y[1].y));
                 }
             } else {
-                for (int i = 0; i < 4; i++) {
-                    if (e + i >= n) break;
+                for (int i = 0; i < UE && e + i < n; i++) {
+                    const float v = (i & 1) ? y[i >> 1].y : y[i >> 1].x;
                     if (BF16OUT)
-                        static_cast<__nv_bfloat16*>(out)[e + i] = __float2bfloat16_rn(y[i]);
+                        static_cast<__nv_bfloat16*>(out)[e + i] = __float2bfloat16_rn(v);
                     else
-                        static_cast<float*>(out)[e + i] = y[i];
+                        static_cast<float*>(out)[e + i] = v;
                 }
             }
         }
@@ -380,9 +420,10 @@ bnbq_status launch_dq(const float* code, const uint8_t* q, const float* absmax, 
     while ((1 << log2B) < B) log2B++;
     int grid = 0;
     auto kern = dequantize_kernel<K, BF16OUT, NESTED>;
-    st = persistent_grid(kern, 256, 0, (n + 3) / 4, 256 * 4, &grid);
+    st = persistent_grid(kern, 256, 0, (n + DqGeom<BF16OUT>::kSpan - 1) / DqGeom<BF16OUT>::kSpan, 256 / 32, &grid);
     if (st != BNBQ_OK) return st;
-    kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags, ns);
+    const bool out16 = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+    kern<<<grid, 256, 0, s>>>(code, q, absmax, n, log2B, out, flags, ns, out16);
     return cuda_status(cudaGetLastError(), "dequantize_kernel launch");
 }
 
