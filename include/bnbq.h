@@ -47,7 +47,7 @@ typedef struct CUstream_st* bnbq_stream_t;
 typedef enum {
     BNBQ_OK = 0,
     BNBQ_EINVAL = 1,       /* an argument is out of range, null, or misaligned */
-    BNBQ_EUNSUPPORTED = 2, /* a valid request this build does not handle */
+    BNBQ_EUNSUPPORTED = 2, /* a valid request this library version does not handle */
     BNBQ_ECUDA = 3         /* a CUDA runtime call failed (see bnbq_last_error) */
 } bnbq_status;
 
