@@ -165,6 +165,13 @@ bnbq_status get_table(const std::vector<StepDesc>& descs, cudaStream_t s, TableE
     for (auto& t : g_tables) {
         if (t.device == dev && t.hash == h && t.host.size() == descs.size() &&
             memcmp(t.host.data(), descs.data(), bytes) == 0) {
+            // order this stream after the table's upload (and its last use), which may have been
+            // issued on another stream (not while the stream is being captured: a capture may not
+            // depend on work recorded outside it)
+            cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+            cudaError_t e = cudaStreamIsCapturing(s, &cap);
+            if (e == cudaSuccess && cap == cudaStreamCaptureStatusNone) e = cudaStreamWaitEvent(s, t.last_use, 0);
+            if (e != cudaSuccess) return cuda_status(e, "cudaStreamWaitEvent(descriptor table)");
             t.tick = ++g_tick;
             *out = &t;
             return BNBQ_OK;
@@ -190,6 +197,7 @@ bnbq_status get_table(const std::vector<StepDesc>& descs, cudaStream_t s, TableE
     memcpy(t.h_pinned, descs.data(), bytes);
     e = cudaEventCreateWithFlags(&t.last_use, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaMemcpyAsync(t.d_table, t.h_pinned, bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaEventRecord(t.last_use, s);
     if (e != cudaSuccess) {
         bnbq_status r = cuda_status(e, "descriptor table upload");
         free_entry(t);

@@ -235,6 +235,31 @@ def test_small_list_other_codebooks(mode, optim):
                      c2.numpy() if two else None, prev)
 
 
+def test_cached_table_used_from_another_stream():
+    """Step t=1 on one stream and t=2 on another, back to back, for the same list: the second
+    call reuses the cached descriptor table and must wait for its upload and for the first step;
+    the result equals the two steps on one stream."""
+    B = 2048
+    ref, c1, c2 = _small_list("adamw", B, torch.bfloat16, 21)
+    got, _, _ = _small_list("adamw", B, torch.bfloat16, 21)
+    bq.bnbq_release()
+    for t in (1, 2):
+        bq.bnbq_step_8bit("adamw", ref, step=t, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP["adamw"])
+    torch.cuda.synchronize()
+    bq.bnbq_release()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    bq.bnbq_step_8bit("adamw", got, step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B,
+                      stream=sa.cuda_stream, **HP["adamw"])
+    bq.bnbq_step_8bit("adamw", got, step=2, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B,
+                      stream=sb.cuda_stream, **HP["adamw"])
+    torch.cuda.synchronize()
+    for r, g in zip(ref, got):
+        for a, b in ((r.p, g.p), (r.state1, g.state1), (r.state2, g.state2), (r.absmax1, g.absmax1),
+                     (r.absmax2, g.absmax2)):
+            if a is not None:
+                assert torch.equal(a, b)
+
+
 def test_zero_gradient_zero_state_stays_zero():
     c1, c2 = _codes()
     n, B = 10000, 2048
