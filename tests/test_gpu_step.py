@@ -303,6 +303,34 @@ def test_optimizer_front_end_matches_direct_call():
     assert [opt.state_bits_for(p) for p in params] == [32, 8, 32]
 
 
+def test_rmsprop_front_end_matches_oracle():
+    """RMSprop8bit over torch parameters: its one state uses the unsigned dynamic code and alpha
+    travels as beta1; each tensor matches the oracle (8-bit for >= 4096 elements, 32-bit below)."""
+    c2 = bq.bnbq_codebook("dynamic_unsigned")
+    params = [torch.nn.Parameter(W.normal(n, 0.02, DEV, "fe-r", i)) for i, n in enumerate([300, 9000])]
+    opt = O.RMSprop8bit(params, lr=1e-3, alpha=0.99, eps=1e-8, weight_decay=0.01)
+    hp = dict(lr=1e-3, beta1=0.99, beta2=0.0, eps=1e-8, weight_decay=0.01)
+    host = [dict(p=parity.to_np(p)) for p in params]
+    for h, p in zip(host, params):
+        n = p.numel()
+        if opt.state_bits_for(p) == 8:
+            h.update(s1=np.zeros(n, np.uint8), a1=np.zeros((n + 2047) // 2048, np.float32))
+        else:
+            h.update(s1=np.zeros(n, np.float32), a1=None)
+    for t in (1, 2, 3):
+        for i, p in enumerate(params):
+            p.grad = W.normal(p.numel(), 1e-3, DEV, "fe-rg", i, t)
+        opt.step()
+        torch.cuda.synchronize()
+        for h, p in zip(host, params):
+            parity.oracle_step_numpy("rmsprop", h["p"], parity.to_np(p.grad), h["s1"], None, h["a1"], None,
+                                     c2.numpy(), None, 2048, hp, t)
+            parity.assert_p_close(parity.to_np(p.detach()), h["p"], "RMSprop front-end p")
+            np.testing.assert_array_equal(parity.to_np(opt.state[p]["state1"]).view(np.uint8 if h["a1"] is not None
+                                                                                    else np.float32), h["s1"])
+    assert [opt.state_bits_for(p) for p in params] == [32, 8]
+
+
 # ---------------------------------------------------------------------------------- full size
 def _sample_ranges(lay, B, picks):
     """(tensor index, first block, last block) ranges to check: whole small tensors, and for big
