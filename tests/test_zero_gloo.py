@@ -114,3 +114,114 @@ def test_two_gloo_ranks_reproduce_single_rank_step(oracle_mod):
             np.testing.assert_array_equal(part["a2"], d["a2"][b0:b1])
             covered += pc.numel
     assert covered == sum(NUMELS)
+
+
+# ------------------------------------------------------------------ the ZeRO-1 exchange, 2 gloo ranks
+OFFS_ALIGN = 16
+
+
+def _flat_offsets(numels):
+    offs, o = [], 0
+    for n in numels:
+        offs.append(o)
+        o += (n + OFFS_ALIGN - 1) // OFFS_ALIGN * OFFS_ALIGN  # gaps between tensors, as in the flat layouts
+    return offs, o
+
+
+def _exchange_inputs(world):
+    rng = np.random.default_rng(7)
+    offs, total = _flat_offsets(NUMELS)
+    p = np.zeros(total, np.float32)
+    for n, o in zip(NUMELS, offs):
+        p[o:o + n] = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    grads = [np.zeros(total, np.float32) for _ in range(world)]
+    for r in range(world):
+        for n, o in zip(NUMELS, offs):
+            grads[r][o:o + n] = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    states = []
+    for n in NUMELS:
+        nb = (n + B - 1) // B
+        states.append(dict(s1=rng.integers(0, 256, n).astype(np.uint8), s2=rng.integers(0, 256, n).astype(np.uint8),
+                           a1=rng.uniform(1e-4, 1e-3, nb).astype(np.float32),
+                           a2=rng.uniform(1e-8, 1e-6, nb).astype(np.float32)))
+    return offs, p, grads, states
+
+
+def _exchange_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        offs, p, grads, states = _exchange_inputs(world)
+        c1, c2 = oracle.code_dynamic_signed(), oracle.code_dynamic_unsigned()
+        ex = zero.ZeroOneExchange(NUMELS, offs, B, world, rank)
+        P = torch.from_numpy(p)
+        g_chunk = ex.reduce_scatter_grads(torch.from_numpy(grads[rank]))
+        mine = []
+        for pc, pv, gv in ex.piece_views(P, g_chunk):
+            st = states[pc.tensor]
+            b0, b1 = pc.first_block, pc.first_block + pc.n_blocks
+            s = {k: np.ascontiguousarray(st[k][pc.start:pc.start + pc.numel]) for k in ("s1", "s2")}
+            a = {k: np.ascontiguousarray(st[k][b0:b1]) for k in ("a1", "a2")}
+            oracle.step_tensor("adamw", pv.numpy(), gv.numpy(), s["s1"], s["s2"], a["a1"], a["a2"], c1, c2, B,
+                               step=5, **HP)
+            mine.append((pc, s, a))
+        ex.all_gather_params(P)
+        q.put((rank, P.numpy().copy(), mine))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_zero1_exchange_two_gloo_ranks_equals_single_rank_step(oracle_mod):
+    """Reduce-scatter of the gradients, a step of each rank's pieces, all-gather of the
+    parameters: every rank ends with the parameters of one single-rank step on the summed
+    gradient, and the pieces' states equal the single-rank states, bit for bit."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    offs, p, grads, states = _exchange_inputs(world)
+    g = grads[0] + grads[1]  # two ranks: the sum is the same in either order
+    c1, c2 = oracle_mod.code_dynamic_signed(), oracle_mod.code_dynamic_unsigned()
+    for n, o, st in zip(NUMELS, offs, states):
+        pv = p[o:o + n]
+        oracle_mod.step_tensor("adamw", pv, np.ascontiguousarray(g[o:o + n]), st["s1"], st["s2"], st["a1"], st["a2"],
+                               c1, c2, B, step=5, **HP)
+    covered = 0
+    for rank, P, mine in results:
+        np.testing.assert_array_equal(P, p)
+        for pc, s, a in mine:
+            st = states[pc.tensor]
+            np.testing.assert_array_equal(s["s1"], st["s1"][pc.start:pc.start + pc.numel])
+            np.testing.assert_array_equal(s["s2"], st["s2"][pc.start:pc.start + pc.numel])
+            np.testing.assert_array_equal(a["a1"], st["a1"][pc.first_block:pc.first_block + pc.n_blocks])
+            np.testing.assert_array_equal(a["a2"], st["a2"][pc.first_block:pc.first_block + pc.n_blocks])
+            covered += pc.numel
+    assert covered == sum(NUMELS)
+
+
+def test_zero1_exchange_ranges():
+    """Each rank's range is contiguous, block-aligned within its tensors, ordered and disjoint;
+    together they cover every tensor; the common chunk holds the longest."""
+    offs, total = _flat_offsets(NUMELS)
+    for world in (1, 2, 3, 8):
+        ranges = [zero.ZeroOneExchange(NUMELS, offs, B, world, r).ranges[r] for r in range(world)]
+        ex = zero.ZeroOneExchange(NUMELS, offs, B, world, 0)
+        assert ranges == ex.ranges
+        nonempty = [(lo, hi) for lo, hi in ranges if hi > lo]
+        assert all(a[1] <= b[0] for a, b in zip(nonempty, nonempty[1:]))
+        assert nonempty[0][0] == 0 and nonempty[-1][1] == offs[-1] + NUMELS[-1]
+        assert ex.chunk >= max(hi - lo for lo, hi in ranges) and ex.chunk % 16 == 0
+        for r, pcs in enumerate(ex.pieces):
+            for pc in pcs:
+                a = offs[pc.tensor] + pc.start
+                assert ranges[r][0] <= a and a + pc.numel <= ranges[r][1]
