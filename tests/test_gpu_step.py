@@ -260,6 +260,30 @@ def test_cached_table_used_from_another_stream():
                 assert torch.equal(a, b)
 
 
+def test_empty_tensors_in_the_list_are_skipped():
+    """Entries with n == 0 (first, middle, last) change nothing and disturb no neighbour."""
+    B = 2048
+    c1, c2 = _codes()
+    full, _, _ = _small_list("adamw", B, torch.bfloat16, 31)
+    ref, _, _ = _small_list("adamw", B, torch.bfloat16, 31)
+
+    def empty():
+        z = torch.empty(0, device=DEV)
+        return bq.TensorState(z, z.to(torch.bfloat16), torch.empty(0, dtype=torch.uint8, device=DEV),
+                              torch.empty(0, dtype=torch.uint8, device=DEV), z, z)
+
+    with_empties = [empty()] + full[:3] + [empty()] + full[3:] + [empty()]
+    bq.bnbq_step_8bit("adamw", with_empties, step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP["adamw"])
+    bq.bnbq_step_8bit("adamw", ref, step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP["adamw"])
+    torch.cuda.synchronize()
+    for r, g in zip(ref, full):
+        for a, b in ((r.p, g.p), (r.state1, g.state1), (r.state2, g.state2)):
+            assert torch.equal(a, b)
+    bq.bnbq_step_8bit("adamw", [empty()], step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP["adamw"])
+    bq.bnbq_step_8bit("adamw", [], step=1, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B, **HP["adamw"])
+    torch.cuda.synchronize()
+
+
 def test_zero_gradient_zero_state_stays_zero():
     c1, c2 = _codes()
     n, B = 10000, 2048
