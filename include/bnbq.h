@@ -21,10 +21,12 @@
  *    device-side check (strictly increasing, finite, within [-1, 1]) makes the kernel write
  *    nothing and sets BNBQ_FLAG_BAD_CODE; non-finite values met while building block scales set
  *    BNBQ_FLAG_NONFINITE.  Read the flags with bnbq_device_flags().
- *  - Blocks have `blocksize` in {256, 2048, 4096} consecutive elements; the last block of a
- *    tensor may be shorter; blocks never span two tensors.  Block b's scale is absmax[b].
+ *  - Blocks have `blocksize` consecutive elements -- 64, 128, 256, 2048 or 4096 for quantize and
+ *    dequantize, 256, 2048 or 4096 for the optimizer step; the last block of a tensor may be
+ *    shorter; blocks never span two tensors.  Block b's scale is absmax[b].
  *  - Alignment (checked; BNBQ_EINVAL if violated): fp32 arrays and fp32 state 16 bytes, bf16
- *    arrays 8 bytes, 8-bit codes 4 bytes, packed NF4 codes 2 bytes, absmax and codebooks 4 bytes.
+ *    arrays 8 bytes, 8-bit codes 4 bytes, packed 4-bit codes 2 bytes, absmax and codebooks 4
+ *    bytes; the nested-scale entry points state their own.
  */
 #ifndef BNBQ_H
 #define BNBQ_H
@@ -63,7 +65,7 @@ typedef enum {
 
 typedef enum {
     BNBQ_CODE_DYNAMIC_SIGNED = 0,   /* 256 values, for m / Lion / momentum state */
-    BNBQ_CODE_DYNAMIC_UNSIGNED = 1, /* 256 values, for Adam's v */
+    BNBQ_CODE_DYNAMIC_UNSIGNED = 1, /* 256 values, for Adam's v and RMSprop's state */
     BNBQ_CODE_NF4 = 2,              /* 16 values */
     BNBQ_CODE_LINEAR = 3,           /* 256 values, -1 + 2k/255 */
     BNBQ_CODE_FP4 = 4               /* 16 values: E2M1 4-bit float / 6, the -0 pattern as +0.25/6 */
