@@ -126,6 +126,20 @@ def _step(opt=0, tensors=None, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), step=1, c1=0x70
     return B.lib().bnbq_step_8bit(opt, arr, len(tensors), ctypes.byref(h), step, c1, c2, Bs, None)
 
 
+def test_step_tensor_count_limits():
+    """More than 2^20 tensors, a negative count, or a NULL list: rejected before any CUDA call."""
+    h = B.CHParams(1e-3, 0.9, 0.999, 1e-8, 0.0)
+    arr = (B.CTensor * 1)(_t())
+    L = B.lib()
+    assert L.bnbq_step_8bit(0, arr, (1 << 20) + 1, ctypes.byref(h), 1, 0x7000, 0x8000, 2048, None) == B.EINVAL
+    assert "2^20" in B.bnbq_last_error()
+    assert L.bnbq_step_8bit(0, arr, -1, ctypes.byref(h), 1, 0x7000, 0x8000, 2048, None) == B.EINVAL
+    assert L.bnbq_step_8bit(0, None, 3, ctypes.byref(h), 1, 0x7000, 0x8000, 2048, None) == B.EINVAL
+    assert L.bnbq_step_8bit(0, None, 0, ctypes.byref(h), 1, 0x7000, 0x8000, 2048, None) == B.OK  # empty list
+    assert L.bnbq_step_8bit(4, arr, 1, ctypes.byref(B.CHParams(1e-3, 1.0, 0.0, 1e-8, 0.0)), 1, 0x7000, None,
+                            2048, None) == B.EINVAL  # RMSprop alpha must be < 1
+
+
 def test_step_argument_checks():
     assert _step(opt=9) == B.EINVAL
     assert _step(step=0) == B.EINVAL
