@@ -153,6 +153,23 @@ def algorithmic_bytes(lay, optim: str, g_bytes: int = 2) -> int:
     return total
 
 
+E2E_SLICES = 4  # with the main list's table, within the library's cache of 8 descriptor tables
+
+
+def e2e_slices(lay, k: int):
+    """Contiguous runs of tensors with about 1/k of the elements each: (first tensor, end tensor,
+    first element, end element of their gradients in the flat buffer)."""
+    n = len(lay.specs)
+    total = sum(s.numel for s in lay.specs)
+    out, i0, acc = [], 0, 0
+    for i, s in enumerate(lay.specs):
+        acc += s.numel
+        if acc * k >= total * (len(out) + 1) or i == n - 1:
+            out.append((i0, i + 1, lay.off[i0], lay.off[i] + s.numel))
+            i0 = i + 1
+    return out
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -433,16 +450,35 @@ def main():
 
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
+        # End to end from host gradients, as a user would drive it: the list is stepped in
+        # E2E_SLICES contiguous slices of tensors (one public bnbq_step_8bit call each); a slice's
+        # gradients are copied host -> device on a side stream and its step starts as soon as they
+        # have landed, so the copies of later slices overlap the steps of earlier ones.  The next
+        # step's copy of a slice waits for that slice's previous step (which reads the buffer).
         g_host = torch.empty(fl.g.numel(), dtype=fl.g.dtype, pin_memory=True)
         g_host.copy_(fl.g)
+        slices = e2e_slices(lay, E2E_SLICES)
+        packed = [(bq.pack_tensor_list(fl.entries[i0:i1]), i1 - i0) for (i0, i1, _, _) in slices]
+        copy_stream = torch.cuda.Stream(dev)
+        landed = [torch.cuda.Event() for _ in slices]
+        stepped = [torch.cuda.Event() for _ in slices]
+        for ev in stepped:
+            ev.record(stream)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
             t += 1
-            fl.g.copy_(g_host, non_blocking=True)
-            fl.step(t, **hp)
+            for k, (i0, i1, a, b) in enumerate(slices):
+                copy_stream.wait_event(stepped[k])
+                with torch.cuda.stream(copy_stream):
+                    fl.g[a:b].copy_(g_host[a:b], non_blocking=True)
+                landed[k].record(copy_stream)
+                stream.wait_event(landed[k])
+                bq.bnbq_step_8bit(optim, packed[k][0], ntensors=packed[k][1], step=t, code1=fl.code1, code2=fl.code2,
+                                  blocksize=lay.blocksize, stream=stream, **hp)
+                stepped[k].record(stream)
             flags |= bq.bnbq_device_flags()  # device -> host read of the step's status word
         e1.record(stream)
         torch.cuda.synchronize()
@@ -453,9 +489,9 @@ def main():
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             e_ms = float(tt.item())
         e2e = {"value": lay.n_params * args.e2e_steps * world / (e_ms / 1e3), "unit": "params/s",
-               "h2d_bytes_per_step": g_host.numel() * g_host.element_size(), "d2h_bytes_per_step": 4,
-               "steps": args.e2e_steps}
-        del g_host
+               "h2d_bytes_per_step": sum(b - a for (_, _, a, b) in slices) * g_host.element_size(),
+               "d2h_bytes_per_step": 4, "steps": args.e2e_steps, "slices": len(slices)}
+        del g_host, packed
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
