@@ -194,3 +194,17 @@ def test_algorithmic_bytes_model():
     lay = W.Layout.build(W.llama7b(), 2048)
     assert algorithmic_bytes(lay, "adamw", g_bytes=2) == 6_607_343_616 * 14 + 3_226_242 * 16 + 131_072_000 * 26
     assert algorithmic_bytes(lay, "lion", g_bytes=2) == 6_607_343_616 * 12 + 3_226_242 * 8 + 131_072_000 * 18
+
+
+def test_e2e_slices_cover_the_list_in_order():
+    """The end-to-end leg of bench.py steps the list in contiguous, element-balanced slices."""
+    from bench import e2e_slices
+    lay = W.Layout.build(W.SHAPES["llama7b"](), 2048)
+    for k in (1, 2, 4, 7):
+        sl = e2e_slices(lay, k)
+        assert sl[0][0] == 0 and sl[-1][1] == len(lay.specs) and len(sl) <= k
+        assert all(a[1] == b[0] and a[3] <= b[2] for a, b in zip(sl, sl[1:]))
+        for i0, i1, a, b in sl:
+            assert a == lay.off[i0] and b == lay.off[i1 - 1] + lay.specs[i1 - 1].numel
+        sizes = [sum(s.numel for s in lay.specs[i0:i1]) for i0, i1, _, _ in sl]
+        assert max(sizes) <= 2 * lay.n_params / k
