@@ -12,7 +12,7 @@ list; each ``step()`` is one call of the CUDA library per parameter group.
 """
 from __future__ import annotations
 
-from typing import Dict, Iterable, List, Optional
+from typing import Dict, List, Optional
 
 import torch
 

@@ -6,7 +6,6 @@ tensors and the result must equal a direct step over the full tensors, bit for b
 multi-rank exchange itself is checked with gloo ranks in test_zero_gloo.py.
 """
 import datetime
-import os
 import socket
 
 import pytest

@@ -10,7 +10,6 @@ SGD, which these tests run in float64 as an independent reference; Lion is pinne
 closed-form special cases.  The 8-bit path is pinned as "dequantize -> the same update ->
 nearest-code requantize" against torch and an exact brute-force nearest code.
 """
-from fractions import Fraction
 
 import numpy as np
 import pytest
