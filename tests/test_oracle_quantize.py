@@ -18,7 +18,7 @@ RNG = np.random.default_rng(12345)
 
 def _codes(o):
     return {"signed": o.code_dynamic_signed(), "unsigned": o.code_dynamic_unsigned(),
-            "nf4": o.code_nf4(), "linear": o.code_linear()}
+            "nf4": o.code_nf4(), "fp4": o.code_fp4(), "linear": o.code_linear()}
 
 
 def _argmin_exact(code, xn):
@@ -57,7 +57,7 @@ def _adversarial_xn(code, rng, n_random):
     return vals
 
 
-@pytest.mark.parametrize("name", ["signed", "unsigned", "nf4", "linear"])
+@pytest.mark.parametrize("name", ["signed", "unsigned", "nf4", "fp4", "linear"])
 def test_nearest_code_exact_bruteforce(oracle_mod, name):
     code = _codes(oracle_mod)[name]
     xs = _adversarial_xn(code, np.random.default_rng(7), 400)
@@ -93,7 +93,7 @@ def _blocks(x, B):
     return [(s, min(n, s + B)) for s in range(0, n, B)]
 
 
-@pytest.mark.parametrize("name", ["signed", "unsigned", "nf4", "linear"])
+@pytest.mark.parametrize("name", ["signed", "unsigned", "nf4", "fp4", "linear"])
 @pytest.mark.parametrize("B", [64, 128, 256, 2048, 4096])
 @pytest.mark.parametrize("bf16", [False, True])
 def test_quantize_blockwise_matches_bruteforce(oracle_mod, name, B, bf16):
@@ -131,7 +131,7 @@ def test_quantize_blockwise_matches_bruteforce(oracle_mod, name, B, bf16):
             assert _is_rounded_mid(code, xn[i]) and got[i] == want[i] - 1
 
 
-@pytest.mark.parametrize("name", ["signed", "unsigned", "linear", "nf4"])
+@pytest.mark.parametrize("name", ["signed", "unsigned", "linear", "nf4", "fp4"])
 def test_round_trip_every_code(oracle_mod, name):
     """P1: a block {code_j * A, A} quantizes back to j, and dequantizes to code_j * A exactly."""
     code = _codes(oracle_mod)[name]
