@@ -212,3 +212,39 @@ def test_sweep_full_size_sampled(log2n, dtype):
                 np.testing.assert_array_equal(parity.to_np(y[b * B:(b + 1) * B]), y_or)
             del a, q, y
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("code_name", ["signed", "nf4"])
+def test_beyond_2p31_elements_sampled(code_name):
+    """Maximum sizes: a bf16 tensor of 2^31 + 4099 elements (element and byte offsets past 32
+    bits, a ragged last block).  Blocks at the start, around element 2^31 and at the end are
+    recomputed by the oracle; every block scale is checked against torch's block maxima."""
+    if torch.cuda.get_device_properties(0).total_memory < 40e9:
+        pytest.skip("needs a GPU with >= 40 GB")
+    n, B = 2 ** 31 + 4099, 4096
+    x = W.normal(n, 1.0, DEV, "huge", code_name).to(torch.bfloat16)
+    code = _codes()[code_name]
+    a, q = bq.bnbq_quantize_blockwise(code.to(DEV), x, B)
+    nb = (n + B - 1) // B
+    full = n // B
+    want_a = x[:full * B].float().view(full, B).abs().amax(dim=1)
+    assert torch.equal(a[:full], want_a)
+    assert float(a[-1]) == float(x[full * B:].float().abs().max())
+    edge = (2 ** 31) // B
+    for b in (0, 1, edge - 1, edge, edge + 1, nb - 2, nb - 1):
+        e0, e1 = b * B, min(n, (b + 1) * B)
+        xs = x[e0:e1].view(torch.int16).cpu().numpy().view(np.uint16)
+        a_or, q_or = oracle.quantize_blockwise(code.numpy(), xs, B)
+        assert parity.to_np(a[b:b + 1]).view(np.uint32)[0] == a_or.view(np.uint32)[0]
+        lo, hi = (e0, e1) if code_name != "nf4" else (e0 // 2, (e1 + 1) // 2)
+        np.testing.assert_array_equal(parity.to_np(q[lo:hi]), q_or)
+    del want_a
+    y = bq.bnbq_dequantize_blockwise(code.to(DEV), q, a, n, B, out_dtype=torch.bfloat16)
+    for b in (0, edge, nb - 1):
+        e0, e1 = b * B, min(n, (b + 1) * B)
+        lo, hi = (e0, e1) if code_name != "nf4" else (e0 // 2, (e1 + 1) // 2)
+        y_or = oracle.dequantize_blockwise(code.numpy(), parity.to_np(q[lo:hi]), parity.to_np(a[b:b + 1]), e1 - e0, B,
+                                           out_bf16=True)
+        np.testing.assert_array_equal(y[e0:e1].view(torch.int16).cpu().numpy().view(np.uint16), y_or)
+    del x, a, q, y
+    torch.cuda.empty_cache()
