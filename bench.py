@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -170,11 +171,27 @@ def e2e_slices(lay, k: int):
     return out
 
 
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'|//[^\n]*|/\*.*?\*/|\s+|[^"\'/\s]+|/', re.S)
+
+
+def _code_only(text: str) -> str:
+    """The source with comments dropped and whitespace runs folded, so that a change to a
+    comment keeps the hash (and the traffic record keyed on it) while any change to code does not."""
+    out = []
+    for tok in _CODE_TOKENS.findall(text):
+        if tok.startswith("//") or tok.startswith("/*") or tok.isspace():
+            out.append("\n" if "\n" in tok else " ")  # line breaks end preprocessor lines
+        else:
+            out.append(tok)
+    return re.sub(r" *\n[\s]*", "\n", re.sub(" +", " ", "".join(out))).strip()
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 
