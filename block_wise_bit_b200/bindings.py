@@ -287,8 +287,8 @@ def bnbq_step_8bit_noalloc(opt: str | int, tensors: Sequence[TensorState] | ctyp
     callers whose device memory all belongs to their own pool, or that must not allocate between
     steps): the descriptor table lives in a fixed array inside the library (at most 4096
     non-empty tensors per call).  All calls on a device share that array, so calls that can
-    overlap on the GPU must be ordered; the first call on a device does a one-time set-up and
-    should come before any stream capture."""
+    overlap on the GPU must be ordered.  Like ``bnbq_step_8bit`` it refuses a stream that is
+    being captured into a CUDA graph."""
     o = OPTIMS[opt] if isinstance(opt, str) else int(opt)
     if isinstance(tensors, ctypes.Array):
         arr, nt = tensors, ntensors

@@ -42,6 +42,17 @@ bnbq_status cuda_status(cudaError_t e, const char* what)
     return fail(BNBQ_ECUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
 }
 
+bnbq_status refuse_capture(cudaStream_t s)
+{
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cap);
+    if (e != cudaSuccess) return cuda_status(e, "cudaStreamIsCapturing");
+    if (cap != cudaStreamCaptureStatusNone)
+        return fail(BNBQ_EUNSUPPORTED, "the stream is being captured: a step's scalars (bias corrections) and "
+                                       "descriptor table belong to one call, so launch it outside the capture");
+    return BNBQ_OK;
+}
+
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
@@ -166,11 +177,8 @@ bnbq_status get_table(const std::vector<StepDesc>& descs, cudaStream_t s, TableE
         if (t.device == dev && t.hash == h && t.host.size() == descs.size() &&
             memcmp(t.host.data(), descs.data(), bytes) == 0) {
             // order this stream after the table's upload (and its last use), which may have been
-            // issued on another stream (not while the stream is being captured: a capture may not
-            // depend on work recorded outside it)
-            cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-            cudaError_t e = cudaStreamIsCapturing(s, &cap);
-            if (e == cudaSuccess && cap == cudaStreamCaptureStatusNone) e = cudaStreamWaitEvent(s, t.last_use, 0);
+            // issued on another stream
+            cudaError_t e = cudaStreamWaitEvent(s, t.last_use, 0);
             if (e != cudaSuccess) return cuda_status(e, "cudaStreamWaitEvent(descriptor table)");
             t.tick = ++g_tick;
             *out = &t;
@@ -503,9 +511,11 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
     sc.wd = hp->weight_decay;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    bnbq_status st = refuse_capture(s);
+    if (st != BNBQ_OK) return st;
     std::lock_guard<std::mutex> lk(g_tab_mu);
     TableEntry* tab = nullptr;
-    bnbq_status st = get_table(descs, s, &tab);
+    st = get_table(descs, s, &tab);
     if (st != BNBQ_OK) return st;
     st = launch_step(opt, tab->d_table, (int)descs.size(), (int)blocks, sc, any8 ? code1 : nullptr,
                      any8 && two ? code2 : nullptr, blocksize, s);

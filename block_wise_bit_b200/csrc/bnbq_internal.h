@@ -12,6 +12,8 @@ namespace bnbq {
 bnbq_status fail(bnbq_status st, const char* fmt, ...);
 // Map a CUDA error to BNBQ_ECUDA with its text (cudaSuccess -> BNBQ_OK).
 bnbq_status cuda_status(cudaError_t e, const char* what);
+// BNBQ_EUNSUPPORTED if `s` is being captured into a CUDA graph (the step entry points refuse it).
+bnbq_status refuse_capture(cudaStream_t s);
 
 // Device-side flag word of the current device (a __device__ variable; its address is taken
 // once per device).

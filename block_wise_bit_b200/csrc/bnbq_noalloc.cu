@@ -148,10 +148,12 @@ extern "C" BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnb
     sc.eps = hp->eps;
     sc.wd = hp->weight_decay;
 
-    StepDesc* d_table = nullptr;
-    bnbq_status st = table_address(&d_table);
-    if (st != BNBQ_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    bnbq_status st = refuse_capture(s);
+    if (st != BNBQ_OK) return st;
+    StepDesc* d_table = nullptr;
+    st = table_address(&d_table);
+    if (st != BNBQ_OK) return st;
     // From pageable host memory: the copy is ordered on `s`, and the host buffer may be reused as
     // soon as the call returns.
     cudaError_t e = cudaMemcpyAsync(d_table, descs, (size_t)nd * sizeof(StepDesc), cudaMemcpyHostToDevice, s);

@@ -189,6 +189,9 @@ typedef struct {
  * absmax = max|state| and the state is requantized by the nearest-code rule above.
  * The library keeps a small per-device cache of uploaded descriptor tables keyed by the list's
  * contents (freed by bnbq_release); a list seen before needs no upload.
+ * A stream that is being captured into a CUDA graph is refused with BNBQ_EUNSUPPORTED before
+ * anything is enqueued: the bias corrections of `step` are kernel arguments and the descriptor
+ * table is rewritten or evicted by later calls, so a replayed capture would not be this call.
  */
 BNBQ_API bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors,
                            const bnbq_hparams* hp, int step, const float* code1,
@@ -203,10 +206,10 @@ BNBQ_API bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int
  * compiled into the library: at most 4096 non-empty tensors per call (256 KiB of device memory
  * on every GPU that loads the library, kept until the process exits); a longer list returns
  * BNBQ_EINVAL.  It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on
- * each device looks up the table's device address and sets the kernel's shared-memory limit; make
- * that first call before capturing any stream.  All calls on a device share the one table and
- * each call rewrites the entries it uses: calls whose work can overlap on the GPU (different
- * streams with no ordering between them) race on it, so order them.
+ * each device looks up the table's device address and sets the kernel's shared-memory limit.  Like
+ * bnbq_step_8bit it refuses a stream that is being captured (BNBQ_EUNSUPPORTED).  All calls on a
+ * device share the one table and each call rewrites the entries it uses: calls whose work can
+ * overlap on the GPU (different streams with no ordering between them) race on it, so order them.
  */
 BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnbq_tensor* list, int ntensors,
                                             const bnbq_hparams* hp, int step, const float* code1,

@@ -17,6 +17,7 @@ import pytest
 import torch
 
 import block_wise_bit_b200 as bq
+from block_wise_bit_b200 import bindings
 from block_wise_bit_b200 import optim as O
 from block_wise_bit_b200 import workloads as W
 
@@ -252,6 +253,42 @@ def test_cached_table_used_from_another_stream():
                       stream=sa.cuda_stream, **HP["adamw"])
     bq.bnbq_step_8bit("adamw", got, step=2, code1=c1.to(DEV), code2=c2.to(DEV), blocksize=B,
                       stream=sb.cuda_stream, **HP["adamw"])
+    torch.cuda.synchronize()
+    for r, g in zip(ref, got):
+        for a, b in ((r.p, g.p), (r.state1, g.state1), (r.state2, g.state2), (r.absmax1, g.absmax1),
+                     (r.absmax2, g.absmax2)):
+            if a is not None:
+                assert torch.equal(a, b)
+
+
+def test_step_refuses_a_capturing_stream():
+    """Both step entry points refuse a stream that is being captured into a CUDA graph with
+    BNBQ_EUNSUPPORTED before enqueuing anything (the capture still ends cleanly), and the same
+    calls outside the capture then step the list as usual."""
+    B = 2048
+    got, c1, c2 = _small_list("adamw", B, torch.bfloat16, 41)
+    ref, _, _ = _small_list("adamw", B, torch.bfloat16, 41)
+    d1, d2 = c1.to(DEV), c2.to(DEV)
+    bq.bnbq_release()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    for fn in (bindings.bnbq_step_8bit, bindings.bnbq_step_8bit_noalloc):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            graph.capture_begin()
+            try:
+                with pytest.raises(bq.BnbqError) as err:
+                    fn("adamw", got, step=1, code1=d1, code2=d2, blocksize=B, stream=s.cuda_stream, **HP["adamw"])
+            finally:
+                graph.capture_end()
+        assert err.value.status == bindings.EUNSUPPORTED
+        assert "captured" in str(err.value)
+        del graph
+    torch.cuda.synchronize()
+    for t in (1, 2):
+        bq.bnbq_step_8bit("adamw", ref, step=t, code1=d1, code2=d2, blocksize=B, **HP["adamw"])
+        bindings.bnbq_step_8bit_noalloc("adamw", got, step=t, code1=d1, code2=d2, blocksize=B, **HP["adamw"])
     torch.cuda.synchronize()
     for r, g in zip(ref, got):
         for a, b in ((r.p, g.p), (r.state1, g.state1), (r.state2, g.state2), (r.absmax1, g.absmax1),
