@@ -32,6 +32,7 @@ def _quantize_pins(o):
             lambda: PQ.test_nearest_code_exact_bruteforce(o, "nf4"),
             lambda: PQ.test_quantize_blockwise_matches_bruteforce(o, "signed", 256, False),
             lambda: PQ.test_quantize_blockwise_matches_bruteforce(o, "nf4", 64, True),
+            lambda: PQ.test_normalisation_is_the_correctly_rounded_quotient(o),
             lambda: PQ.test_round_trip_every_code(o, "signed"),
             lambda: PQ.test_nf4_nibble_order(o),
             lambda: PQ.test_dequantize_bf16_matches_torch_rounding(o),
@@ -42,8 +43,11 @@ def _step_pins(o):
     return [lambda: PS.test_adamw_32bit_matches_torch(o, 0.01), lambda: PS.test_adamw_first_step_closed_form(o),
             lambda: PS.test_adam_l2_matches_torch(o), lambda: PS.test_momentum_matches_torch_sgd(o, 0.01),
             lambda: PS.test_momentum_first_step(o), lambda: PS.test_lion_sign_update(o),
+            lambda: PS.test_lion_decay_uses_the_old_parameter(o),
             lambda: PS.test_rmsprop_matches_torch(o, 0.01), lambda: PS.test_rmsprop_first_step_closed_form(o),
-            lambda: PS.test_8bit_first_step_equals_32bit(o)]
+            lambda: PS.test_rmsprop_8bit_step_matches_torch(o), lambda: PS.test_8bit_first_step_equals_32bit(o),
+            lambda: PS.test_8bit_step_from_quantized_state_matches_torch(o),
+            lambda: PS.test_zero_gradient_zero_state_stays(o), lambda: PS.test_bf16_gradients_are_widened_exactly(o)]
 
 
 def _nested_pins(o):
@@ -81,6 +85,20 @@ MUTANTS = {
                                     "float s = (c > 0.0f) ? -1.0f : ((c < 0.0f) ? 1.0f : 0.0f);")]),
     "momentum with dampening": ("step", [("float m1 = d->b1 * (*m) + g;", "float m1 = d->b1 * (*m) + d->omb1 * g;")]),
     "RMSprop eps inside the root": ("step", [("float denom = sqrtf(v1) + d->eps;", "float denom = sqrtf(v1 + d->eps);")]),
+    "normalisation by a rounded reciprocal": ("quantize", [("float xn = (absmax == 0.0f) ? 0.0f : x / absmax;",
+                                                            "float xn = (absmax == 0.0f) ? 0.0f : x * (1.0f / absmax);")]),
+    "requantize with the old block scale": ("step", [("float a1 = block_absmax(mbuf, len);\n            absmax1[b] = a1;",
+                                                      "float a1 = absmax1[b];")]),
+    "state dequantized with the next block's scale": ("step", [("mbuf[i] = code1[((const uint8_t*)s1)[e]] * absmax1[b];",
+                                                                "mbuf[i] = code1[((const uint8_t*)s1)[e]] * absmax1[(b + 1 < nb) ? b + 1 : b];")]),
+    "Lion state becomes the interpolation c": ("step", [("*m = d->b2 * (*m) + d->omb2 * g;", "*m = c;")]),
+    "Lion decay applied after the sign step": ("step", [("pv = pv * d->decay;\n        pv = pv - d->lr * s;",
+                                                         "pv = pv - d->lr * s;\n        pv = pv * d->decay;")]),
+    "second-moment correction uses beta1": ("step", [("d.sqrt_bc2 = (float)sqrt(1.0 - pow(b2, (double)t));",
+                                                      "d.sqrt_bc2 = (float)sqrt(1.0 - pow(b1, (double)t));")]),
+    "bf16 widening drops the sign": ("step", [("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)(h & 0x7fffu) << 16;")]),
+    "RMSprop alpha and 1 - alpha swapped": ("step", [("float v1 = d->b1 * (*m) + (d->omb1 * g) * g;",
+                                                      "float v1 = d->omb1 * (*m) + (d->b1 * g) * g;")]),
     "nested mean divides by nb + 1": ("nested", [("return (float)(total / (double)nb);", "return (float)(total / (double)(nb + 1));")]),
     "nested scales not centred": ("nested", [("centred[i] = absmax[i] - mean;", "centred[i] = absmax[i];")]),
     "nested rebuild adds before multiplying": ("nested", [("out[i] = code2[qabs[i]] * absmax2[i / ORACLE_NEST_B] + offset;",

@@ -131,6 +131,35 @@ def test_quantize_blockwise_matches_bruteforce(oracle_mod, name, B, bf16):
             assert _is_rounded_mid(code, xn[i]) and got[i] == want[i] - 1
 
 
+def test_normalisation_is_the_correctly_rounded_quotient(oracle_mod):
+    """x / absmax is one binary32 division (numpy's float32 division is IEEE's correctly rounded
+    one), not x times a rounded reciprocal of absmax.  For scales whose reciprocal is inexact the
+    inputs are chosen where the two normalisations fall on opposite sides of a decision
+    midpoint.  The decision rule itself (xn above the binary32 midpoint of two neighbouring
+    codes, ties to the lower code) is pinned against exact nearest-code brute force above; here
+    it is taken as given, so that only the quotient is under test."""
+    code = oracle_mod.code_dynamic_signed()
+    c64 = code.astype(np.float64)
+    mid32 = np.float32((c64[:-1] + c64[1:]) / 2)
+
+    def decide(xn):
+        return np.searchsorted(mid32, xn, side="left")  # number of midpoints strictly below xn
+
+    for a in (3.0, 7.0, 0.3):
+        a32 = np.float32(a)
+        r32 = np.float32(1) / a32
+        picks = []
+        for m in mid32:
+            near = (np.float32(m * a32).view(np.int32) + np.arange(-64, 65)).astype(np.int32).view(np.float32)
+            near = near[np.abs(near) < a32]
+            picks.extend(near[decide(near / a32) != decide(near * r32)].tolist())
+        assert len(picks) >= 40
+        x = np.array(picks + [float(a32)], np.float32)  # the last element sets the block's absmax
+        absmax, q = oracle_mod.quantize_blockwise(code, x, 4096)
+        assert absmax[0] == a32
+        np.testing.assert_array_equal(q.astype(np.int64), decide(x / a32))
+
+
 @pytest.mark.parametrize("name", ["signed", "unsigned", "linear", "nf4", "fp4"])
 def test_round_trip_every_code(oracle_mod, name):
     """P1: a block {code_j * A, A} quantizes back to j, and dequantizes to code_j * A exactly."""

@@ -154,6 +154,27 @@ def test_lion_sign_update(oracle_mod):
     np.testing.assert_allclose(m, m64, rtol=1e-6, atol=1e-12)
 
 
+def test_lion_decay_uses_the_old_parameter(oracle_mod):
+    """Lion as X. Chen et al., "Symbolic Discovery of Optimization Algorithms", Algorithm 2:
+    theta <- theta - lr * (sign(c) + wd * theta), the decay taken on the parameter before the
+    sign step.  With lr * wd = 0.1 a decay applied after the sign step would be off by
+    lr^2 * wd = 0.01 per element."""
+    n, lr, wd = 5000, 0.1, 1.0
+    rng = np.random.default_rng(16)
+    p0 = rng.standard_normal(n).astype(np.float32)
+    m0 = rng.standard_normal(n).astype(np.float32)
+    g = rng.standard_normal(n).astype(np.float32)
+    p, m = p0.copy(), m0.copy()
+    oracle_mod.step_tensor("lion", p, g, m, None, None, None, None, None, 2048, step=1,
+                           lr=lr, beta1=0.9, beta2=0.99, eps=0.0, weight_decay=wd)
+    c64 = _f(0.9) * m0.astype(np.float64) + (1 - _f(0.9)) * g
+    clear = np.abs(c64) > 1e-6
+    assert clear.mean() > 0.99
+    want = p0.astype(np.float64) - _f(lr) * (np.sign(c64) + _f(wd) * p0.astype(np.float64))
+    err = np.abs(p[clear] - want[clear])
+    assert np.all(err <= 4e-6 * (1 + np.abs(want[clear]))), err.max()
+
+
 @pytest.mark.parametrize("wd", [0.0, 1e-2])
 def test_rmsprop_matches_torch(oracle_mod, wd):
     """RMSprop (named by the page "bitsandbytes深度解析", section "优化器模块深度分析", as
