@@ -36,6 +36,7 @@ def _quantize_pins(o):
             lambda: PQ.test_round_trip_every_code(o, "signed"),
             lambda: PQ.test_nf4_nibble_order(o),
             lambda: PQ.test_dequantize_bf16_matches_torch_rounding(o),
+            lambda: PQ.test_dequantize_bf16_ties_to_even(o),
             lambda: PQ.test_error_bound(o, "signed")]
 
 
@@ -85,6 +86,11 @@ MUTANTS = {
                                     "float s = (c > 0.0f) ? -1.0f : ((c < 0.0f) ? 1.0f : 0.0f);")]),
     "momentum with dampening": ("step", [("float m1 = d->b1 * (*m) + g;", "float m1 = d->b1 * (*m) + d->omb1 * g;")]),
     "RMSprop eps inside the root": ("step", [("float denom = sqrtf(v1) + d->eps;", "float denom = sqrtf(v1 + d->eps);")]),
+    "bf16 narrowing rounds ties up": ("quantize", [("u += 0x7fffu + lsb;", "u += 0x8000u + 0u * lsb;")]),
+    "block absmax of signed values": ("quantize", [("float m = fabsf(v[i]);", "float m = v[i];")]),
+    "step leaves the last element of a ragged block": ("step", [(
+        "int64_t len = (n - start < B) ? (n - start) : B;\n        /* 1. load",
+        "int64_t len = (n - start < B) ? (n - start - 1) : B;\n        /* 1. load")]),
     "normalisation by a rounded reciprocal": ("quantize", [("float xn = (absmax == 0.0f) ? 0.0f : x / absmax;",
                                                             "float xn = (absmax == 0.0f) ? 0.0f : x * (1.0f / absmax);")]),
     "requantize with the old block scale": ("step", [("float a1 = block_absmax(mbuf, len);\n            absmax1[b] = a1;",

@@ -286,6 +286,22 @@ def test_dequantize_bf16_matches_torch_rounding(oracle_mod):
     np.testing.assert_array_equal(y / np.repeat(absmax2, B)[:n], code[q])
 
 
+def test_dequantize_bf16_ties_to_even(oracle_mod):
+    """bf16 output rounds to nearest with ties to even, as torch's float32 -> bfloat16
+    conversion does.  A codebook made of exact halfway cases (low 16 bits 0x8000) with both
+    parities of the kept bits, dequantized with absmax 1, puts every tie through the narrowing."""
+    his = np.arange(0x3E00, 0x3E00 + 127, dtype=np.uint32)  # both parities, values in [0.125, 0.25)
+    ties = ((his << 16) | 0x8000).view(np.float32)
+    code = np.sort(np.concatenate([ties, -ties, np.float32([0.0, 1.0])]).astype(np.float32))
+    assert code.size == 256 and np.all(np.diff(code) > 0)
+    q = np.arange(256, dtype=np.uint8)
+    y = oracle_mod.dequantize_blockwise(code, q, np.ones(1, np.float32), 256, 256, out_bf16=True)
+    want = torch.from_numpy(code).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(y, want)
+    kept = (code.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.any(want == kept) and np.any(want != kept)  # some ties stay, some round away
+
+
 def test_rejects_bad_arguments(oracle_mod):
     code = oracle_mod.code_dynamic_signed()
     with pytest.raises(ValueError):
