@@ -81,8 +81,9 @@ __device__ __forceinline__ Pairs make_pairs(const StepScalars& sc)
 
 // One pair of elements of the update.  Every binary32 operation is rounded on its own, in the
 // order the header documents; p - c*u is formed as p + (-c)*u, which rounds identically.
-// sqrt(v)/sqrt(1-b2^t) uses the FMA quotient: the host guarantees sqrt(1-b2^t) lies in
-// [2^-12, 1] (any binary32 b2 < 1), and sqrt(v) is 0 or at least 2^-75, so the quotient is exact.
+// sqrt(v)/sqrt(1-b2^t) uses the FMA quotient: the host rejects sqrt(1-b2^t) outside [2^-60, 1]
+// (any binary32 b2 < 1 gives at least 2^-12), and sqrt(v) is 0 or at least 2^-75, so the
+// quotient is the correctly rounded one.
 template <int OPT>
 __device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, float2& p, float2 g,
                                         float2& m, float2& v)

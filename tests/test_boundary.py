@@ -208,3 +208,19 @@ def test_e2e_slices_cover_the_list_in_order():
             assert a == lay.off[i0] and b == lay.off[i1 - 1] + lay.specs[i1 - 1].numel
         sizes = [sum(s.numel for s in lay.specs[i0:i1]) for i0, i1, _, _ in sl]
         assert max(sizes) <= 2 * lay.n_params / k
+
+
+def test_traffic_record_hash_ignores_comments_only():
+    """bench.py keys the committed ncu traffic on a hash of the step kernel's sources with
+    comments removed and spaces folded (line breaks kept): editing a comment keeps the key,
+    editing code changes it."""
+    from bench import _code_only
+    src = ('#include "a.h"\n#define N 16 // elements\nint f(int x) { /* twice */ return 2 * x; }\n'
+           'const char* s = "a // b /* c */";\nchar c = \'/\';\n')
+    same = ('#include "a.h"\n\n// a comment line\n#define N 16   // per thread\nint f(int x) {  return 2 * x; }'
+            '\nconst char* s = "a // b /* c */";\nchar c = \'/\';  /* slash */\n')
+    assert _code_only(src) == _code_only(same)
+    assert _code_only(src) != _code_only(src.replace("2 * x", "3 * x"))
+    assert _code_only(src) != _code_only(src.replace("#define N 16 // elements\n", "#define N 16 int\n"))
+    assert "a // b /* c */" in _code_only(src)  # string contents are code
+    assert _code_only("#define A 1\nint y;") != _code_only("#define A 1 int y;")  # line ends kept
