@@ -8,6 +8,7 @@ import socket
 import numpy as np
 import torch
 import torch.distributed as dist
+from hypothesis import given, settings, strategies as st
 import torch.multiprocessing as mp
 
 from block_wise_bit_b200 import zero
@@ -84,6 +85,28 @@ def test_partition_covers_every_block_once_and_balances():
         assert len(seen) == sum((n + B - 1) // B for n in NUMELS)
         loads = [sum(pc.numel for pc in pieces) for pieces in shards]
         assert max(loads) - min(loads) <= 2 * B or world > len(seen)
+
+
+@settings(max_examples=300, deadline=None)
+@given(numels=st.lists(st.integers(0, 20000), max_size=12), bs=st.sampled_from([256, 2048, 4096]),
+       world=st.integers(1, 9))
+def test_partition_properties_on_random_lists(numels, bs, world):
+    """Any list (empty tensors included), blocksize and world size: every block lands on exactly
+    one rank, ranks hold consecutive runs of the list's blocks in rank order, pieces are
+    block-aligned, and no rank holds more than its equal share plus one block."""
+    shards = zero.partition(numels, bs, world)
+    assert len(shards) == world
+    order = [(t, b) for t, n in enumerate(numels) for b in range((n + bs - 1) // bs)]
+    got = []
+    for pieces in shards:
+        for pc in pieces:
+            assert pc.n_blocks >= 1 and pc.start == pc.first_block * bs
+            assert pc.numel == min(numels[pc.tensor], (pc.first_block + pc.n_blocks) * bs) - pc.start
+            got += [(pc.tensor, b) for b in range(pc.first_block, pc.first_block + pc.n_blocks)]
+    assert got == order
+    total = sum(numels)
+    for pieces in shards:
+        assert sum(pc.numel for pc in pieces) < total / world + bs or total == 0
 
 
 def test_two_gloo_ranks_reproduce_single_rank_step(oracle_mod):
@@ -224,3 +247,27 @@ def test_zero1_exchange_ranges():
             for pc in pcs:
                 a = offs[pc.tensor] + pc.start
                 assert ranges[r][0] <= a and a + pc.numel <= ranges[r][1]
+
+
+@settings(max_examples=200, deadline=None)
+@given(numels=st.lists(st.integers(0, 20000), min_size=1, max_size=10), bs=st.sampled_from([256, 2048]),
+       world=st.integers(1, 8))
+def test_zero1_exchange_ranges_on_random_lists(numels, bs, world):
+    """Random lists: the ranks' flat ranges are ordered and disjoint, each holds exactly its own
+    pieces, every element of every tensor falls in some rank's range, and the common chunk holds
+    the longest range (so the padded reduce-scatter and all-gather move every element once)."""
+    offs, _ = _flat_offsets(numels)
+    ex = zero.ZeroOneExchange(numels, offs, bs, world, 0)
+    nonempty = [(lo, hi) for lo, hi in ex.ranges if hi > lo]
+    assert all(a[1] <= b[0] for a, b in zip(nonempty, nonempty[1:]))
+    assert ex.chunk % 16 == 0 and ex.chunk >= max([hi - lo for lo, hi in ex.ranges] + [1])
+    owner = {}
+    for r, pcs in enumerate(ex.pieces):
+        for pc in pcs:
+            a = offs[pc.tensor] + pc.start
+            assert ex.ranges[r][0] <= a and a + pc.numel <= ex.ranges[r][1]
+            owner.setdefault(pc.tensor, []).append((pc.start, pc.start + pc.numel))
+    for t, n in enumerate(numels):
+        spans = sorted(owner.get(t, []))
+        assert sum(e - s for s, e in spans) == n
+        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:])) and (not spans or spans[0][0] == 0)
