@@ -106,6 +106,8 @@ MUTANTS = {
     "RMSprop alpha and 1 - alpha swapped": ("step", [("float v1 = d->b1 * (*m) + (d->omb1 * g) * g;",
                                                       "float v1 = d->omb1 * (*m) + (d->b1 * g) * g;")]),
     "nested mean divides by nb + 1": ("nested", [("return (float)(total / (double)nb);", "return (float)(total / (double)(nb + 1));")]),
+    "nested mean accumulated in binary32": ("nested", [("        double s = 0.0;", "        float s = 0.0f;")]),
+    "nested offset not stored": ("nested", [("    *offset = mean;", "    *offset = 0.0f;")]),
     "nested scales not centred": ("nested", [("centred[i] = absmax[i] - mean;", "centred[i] = absmax[i];")]),
     "nested rebuild adds before multiplying": ("nested", [("out[i] = code2[qabs[i]] * absmax2[i / ORACLE_NEST_B] + offset;",
                                                           "out[i] = (code2[qabs[i]] + offset) * absmax2[i / ORACLE_NEST_B];")]),
