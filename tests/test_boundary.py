@@ -8,6 +8,7 @@
 import ctypes
 import os
 import re
+import subprocess
 
 import numpy as np
 import pytest
@@ -224,3 +225,42 @@ def test_traffic_record_hash_ignores_comments_only():
     assert _code_only(src) != _code_only(src.replace("#define N 16 // elements\n", "#define N 16 int\n"))
     assert "a // b /* c */" in _code_only(src)  # string contents are code
     assert _code_only("#define A 1\nint y;") != _code_only("#define A 1 int y;")  # line ends kept
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "bnbq.h"
+
+int main(void)
+{
+    static const bnbq_code_kind kinds[] = {BNBQ_CODE_DYNAMIC_SIGNED, BNBQ_CODE_DYNAMIC_UNSIGNED, BNBQ_CODE_NF4,
+                                           BNBQ_CODE_FP4, BNBQ_CODE_LINEAR};
+    float code[256];
+    printf("%s\n", bnbq_version());
+    for (unsigned k = 0; k < sizeof kinds / sizeof kinds[0]; k++) {
+        int K = bnbq_code_size(kinds[k]);
+        if (bnbq_codebook(kinds[k], code) != K || bnbq_check_codebook(code, K) != BNBQ_OK) return 1;
+        for (int j = 0; j < K; j++) printf("%a%c", code[j], j + 1 < K ? ' ' : '\n');
+    }
+    code[1] = code[0];  /* not strictly increasing */
+    if (bnbq_check_codebook(code, 16) != BNBQ_EINVAL || bnbq_last_error()[0] == '\0') return 2;
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C11 program that includes only bnbq.h and links the shared library builds with warnings
+    as errors, and its host-side calls give the same codebooks as the Python binding."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(B.library_path())
+    cuda_lib = "/usr/local/cuda/lib64"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), "-L", libdir, "-lbnbq", f"-Wl,-rpath,{libdir}:{cuda_lib}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    assert out[0] == B.bnbq_version()
+    for line, kind in zip(out[1:6], ["dynamic_signed", "dynamic_unsigned", "nf4", "fp4", "linear"]):
+        got = np.array([float.fromhex(t) for t in line.split()], np.float32)
+        np.testing.assert_array_equal(got, B.bnbq_codebook(kind).numpy())
