@@ -7,8 +7,8 @@
  * "《通过块级量化的8位优化器》翻译与解读".  Stateful optimizers keep per-parameter statistics
  * (momentum's smoothed gradient sum, Adam's smoothed sum and squared sum); the abstract stores
  * them in 8 bits by block-wise quantization -- the tensor is cut into blocks that are quantized
- * independently, each in parallel -- with a dynamic (non-linear) code that is precise for
- * both large and small magnitudes.  NF4 is the 16-value 4-bit type of the page "Bitsandbytes"
+ * independently, each in parallel -- with a dynamic (non-linear) code whose relative error
+ * stays small across many orders of magnitude.  NF4 is the 16-value 4-bit type of the page "Bitsandbytes"
  * (transformers docs), section "Normal Float 4 (NF4)".
  *
  * Conventions for every entry point:

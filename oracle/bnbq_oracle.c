@@ -15,8 +15,8 @@
 /* ------------------------------------------------------------------------------------
  * Codebooks.
  *
- * [BWQ] names "dynamic quantization, a non-linear quantization that is precise for both
- * large and small magnitude values" and gives no values.  Reading taken: the dynamic tree
+ * [BWQ] names dynamic quantization, a non-linear code meant to keep small and large
+ * magnitudes alike accurate, and gives no values.  Reading taken: the dynamic tree
  * of the same paper -- a magnitude is 10^-E * f where E counts leading zero bits, one
  * indicator bit follows, and the remaining bits select one of 2^nE equal fraction bins of
  * (0.1, 1]; the bin's upper edge is used, so the largest code is exactly 1.

@@ -41,9 +41,9 @@
  * Floating point: IEEE binary32, round to nearest even, every operation rounded on its own
  * (built with -ffp-contract=off, no -ffast-math), division and sqrtf correctly rounded,
  * subnormals kept.  Scalars derived from the hyper-parameters are formed in double and
- * rounded once to float.  The abstract fixes the optimizer's update precision at 32 bits
- * ("8-bit statistics while maintaining the performance levels of 32-bit optimizer
- * states"), so the update and every quantization decision are taken in binary32.
+ * rounded once to float.  Per [BWQ]'s abstract only the stored optimizer statistics are 8-bit
+ * and the optimizer is meant to behave as its 32-bit counterpart, so the update and every
+ * quantization decision are taken in binary32.
  *
  * Parity status: every function here is pinned by tests/test_oracle_*.py against exact
  * rational arithmetic, scipy's normal distribution, or torch.optim; none is unpinned.
