@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -339,6 +340,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="8-bit elements in the CPU oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="wall time the CPU baseline aims for (consecutive oracle steps over the sample)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -513,7 +516,10 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_threads()
-        r, dt, sample = oracle_rate(shape, optim, hp, args.cpu_sample, threads, 1)
+        r, dt, sample = oracle_rate(shape, optim, hp, args.cpu_sample, threads, 1)  # also warms up
+        if dt < args.cpu_seconds:
+            k = max(2, math.ceil(args.cpu_seconds / max(dt, 1e-3)))
+            r, dt, sample = oracle_rate(shape, optim, hp, args.cpu_sample, threads, k)
         cpu = {"value": r, "unit": "params/s", "cores": threads, "kind": "oracle", "sample": sample,
                "seconds": round(dt, 2)}
 
