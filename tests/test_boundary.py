@@ -9,6 +9,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -264,3 +265,20 @@ def test_header_is_plain_c_and_links(tmp_path):
     for line, kind in zip(out[1:6], ["dynamic_signed", "dynamic_unsigned", "nf4", "fp4", "linear"]):
         got = np.array([float.fromhex(t) for t in line.split()], np.float32)
         np.testing.assert_array_equal(got, B.bnbq_codebook(kind).numpy())
+
+
+def test_bench_reference_arm_prints_the_contract_line():
+    """``bench.py --impl reference`` (the oracle timed on the host) prints one JSON line with the
+    benchmark's metric, unit and workload, the oracle as cpu_baseline and a host-only e2e."""
+    import json
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                          "--warmup", "3", "--cpu-sample", "65536"], capture_output=True, text=True, check=True,
+                         cwd=ROOT, timeout=600).stdout.strip().split("\n")
+    line = json.loads(out[-1])
+    assert line["impl"] == "reference" and line["unit"] == "params/s" and line["higher_is_better"] is True
+    assert line["steps"] == 2 and line["warmup"] == 3 and line["n_gpus"] == 1 and line["value"] > 0
+    assert line["config"]["workload"] == "llama7b_adamw8bit" and line["config"]["params"] == 6738415616
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "params/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
