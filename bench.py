@@ -328,6 +328,23 @@ def cpu_threads() -> int:
         return os.cpu_count() or 1
 
 
+# ----------------------------------------------------------------------------- rank aggregation
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's time; every rank calls this at the same point (one all-reduce)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(params_per_rank: int, steps: int, world: int, ms: float) -> float:
+    """Parameters stepped by all ranks per second, over the slowest rank's time."""
+    return params_per_rank * steps * world / (ms / 1e3)
+
+
 # -------------------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -451,12 +468,9 @@ def main():
     total_ms = ev0.elapsed_time(ev1)
     launch_ms = [a.elapsed_time(b) for a, b in zip(k_start, k_end)]
     avg_launch_ms = sum(launch_ms) / len(launch_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_per_step = total_ms / args.steps
-    value = lay.n_params * args.steps * world / (total_ms / 1e3)
+    value = whole_job_rate(lay.n_params, args.steps, world, total_ms)
     flags = bq.bnbq_device_flags(clear=True)
 
     alg = algorithmic_bytes(lay, optim, 2)
@@ -504,11 +518,8 @@ def main():
         torch.cuda.synchronize()
         barrier()
         e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": lay.n_params * args.e2e_steps * world / (e_ms / 1e3), "unit": "params/s",
+        e_ms = max_over_ranks(e_ms, dev, world)
+        e2e = {"value": whole_job_rate(lay.n_params, args.e2e_steps, world, e_ms), "unit": "params/s",
                "h2d_bytes_per_step": sum(b - a for (_, _, a, b) in slices) * g_host.element_size(),
                "d2h_bytes_per_step": 4, "steps": args.e2e_steps, "slices": len(slices)}
         del g_host, packed
