@@ -1,8 +1,8 @@
 """Pins for the oracle's codebooks (CPU only).
 
-The pages fix only that the code is "dynamic": non-linear and precise for both large and small
-magnitudes ([BWQ] abstract, "8-bit Optimizers via Block-wise Quantization", as quoted on the
-blog.csdn.net bitsandbytes guide, section 2), and that NF4 is a 4-bit type fitted to normally
+The pages fix only that the code is dynamic: a non-linear code that keeps small and large
+magnitudes alike accurate ([BWQ] abstract, "8-bit Optimizers via Block-wise Quantization", as
+reproduced on the blog.csdn.net bitsandbytes guide, section 2), and that NF4 is a 4-bit type fitted to normally
 distributed weights ("Bitsandbytes" transformers docs, section "Normal Float 4 (NF4)").  The
 construction read from them (dynamic tree; NF4 from normal quantiles) is pinned here by
 properties that do not restate the oracle's formulas: counts per decade, equal spacing within

@@ -1,9 +1,9 @@
 """Pins for the oracle's optimizer step (CPU only).
 
-The abstract of "8-bit Optimizers via Block-wise Quantization" (quoted on the blog.csdn.net
+The abstract of "8-bit Optimizers via Block-wise Quantization" (reproduced on the blog.csdn.net
 bitsandbytes guide, section 2) names the stateful optimizers -- SGD with momentum (smoothed
-sum) and Adam (smoothed and squared sums) -- and says the 8-bit optimizers are a drop-in
-replacement that keeps 32-bit performance.  The page "bitsandbytes深度解析", section
+sum) and Adam (smoothed and squared sums) -- and presents the 8-bit versions as substitutes
+that need no other change and behave as the 32-bit ones.  The page "bitsandbytes深度解析", section
 "优化器模块深度分析", lists AdamW8bit, Adam8bit, SGD8bit and Lion8bit.  So with quantization
 out of the way (32-bit state) the oracle's step must agree with torch.optim's AdamW, Adam and
 SGD, which these tests run in float64 as an independent reference; Lion is pinned by its
