@@ -24,7 +24,7 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "bnbq_oracle.c")
 def _codebook_pins(o):
     return [lambda: PC.test_unsigned_dynamic_structure(o), lambda: PC.test_signed_dynamic_structure(o),
             lambda: PC.test_dynamic_codes_correctly_rounded(o), lambda: PC.test_nf4_normal_quantiles(o),
-            lambda: PC.test_fp4_e2m1_values(o)]
+            lambda: PC.test_fp4_e2m1_values(o), lambda: PC.test_linear_code(o)]
 
 
 def _quantize_pins(o):
@@ -73,6 +73,13 @@ MUTANTS = {
     "dynamic code on the lower bin edge": ("codebooks", [("(double)((1 << nE) + 9 * (k + 1))", "(double)((1 << nE) + 9 * k)")]),
     "NF4 offset delta = 1/30": ("codebooks", [("const double delta = 0.5 * (1.0 / 30.0 + 1.0 / 32.0);",
                                                "const double delta = 1.0 / 30.0;")]),
+    "NF4 negative half spaced like the positive half": ("codebooks", [(
+        "double prob = delta + (0.5 - delta) * (double)k / 7.0;", "double prob = delta + (0.5 - delta) * (double)k / 8.0;")]),
+    "NF4 positive half not scaled to 1": ("codebooks", [(
+        "double prob = 0.5 + (0.5 - delta) * (double)k / 8.0;\n        out[c++] = (float)(normal_quantile(prob) / scale);",
+        "double prob = 0.5 + (0.5 - delta) * (double)k / 8.0;\n        out[c++] = (float)(normal_quantile(prob));")]),
+    "FP4 exponent without its bias": ("codebooks", [("ldexp(1.0 + 0.5 * (double)f, e - 1)", "ldexp(1.0 + 0.5 * (double)f, e)")]),
+    "linear code steps by 2/256": ("codebooks", [("(float)(-1.0 + 2.0 * (double)k / 255.0)", "(float)(-1.0 + 2.0 * (double)k / 256.0)")]),
     "FP4 spare pattern duplicates a code": ("codebooks", [("out[c++] = (float)(0.25 / 6.0);", "out[c++] = (float)(0.5 / 6.0);")]),
     "Adam m drops (1 - b1)": ("step", [("float m1 = d->b1 * (*m) + d->omb1 * g;", "float m1 = d->b1 * (*m) + g;")]),
     "Adam v not squared": ("step", [("float v1 = d->b2 * (*v) + (d->omb2 * g) * g;", "float v1 = d->b2 * (*v) + (d->omb2 * g);")]),
