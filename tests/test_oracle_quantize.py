@@ -12,6 +12,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 RNG = np.random.default_rng(12345)
 
@@ -308,3 +309,40 @@ def test_rejects_bad_arguments(oracle_mod):
         oracle_mod.quantize_blockwise(code, np.zeros(10, np.float32), 1000)
     with pytest.raises(ValueError):
         oracle_mod.quantize_blockwise(code[:100], np.zeros(10, np.float32), 256)
+
+
+_VALUES = st.one_of(st.floats(-1e4, 1e4, width=32, allow_subnormal=True),
+                    st.sampled_from([0.0, -0.0, 1e-45, -1e-45, 3.4e38, -3.4e38, 1.0, -1.0]))
+
+
+@settings(max_examples=150, deadline=None)
+@given(x=st.lists(_VALUES, max_size=300), B=st.sampled_from([64, 128, 256]),
+       name=st.sampled_from(["signed", "nf4", "fp4", "unsigned"]))
+def test_quantize_random_blocks_match_bruteforce(oracle_mod, x, B, name):
+    """Random lengths (empty and ragged included), blocksizes, codebooks and values (zeros,
+    subnormals, huge values, exact codes): each block's scale is its largest magnitude and each
+    element takes the exact nearest code of its binary32 quotient (ties and rounded midpoints to
+    the lower code), packed two per byte for 4-bit codes."""
+    code = _codes(oracle_mod)[name]
+    xs = np.array(x, np.float32)
+    if code.min() >= 0:
+        xs = np.abs(xs)
+    n = xs.size
+    absmax, q = oracle_mod.quantize_blockwise(code, xs, B)
+    assert absmax.shape == ((n + B - 1) // B,)
+    if len(code) == 16:
+        assert q.size == (n + 1) // 2
+        qi = np.empty(n, np.int64)
+        qi[0::2] = q[: (n + 1) // 2] >> 4
+        qi[1::2] = (q & 0xF)[: n // 2]
+    else:
+        qi = q.astype(np.int64)
+    for b, (s, e) in enumerate(_blocks(xs, B)):
+        blk = xs[s:e]
+        a = np.max(np.abs(blk))
+        assert absmax[b] == a
+        xn = blk / a if a > 0 else np.zeros_like(blk)
+        for i in range(e - s):
+            want = _argmin_exact(code, xn[i])
+            got = int(qi[s + i])
+            assert got == want or (_is_rounded_mid(code, xn[i]) and got == want - 1), (b, i, xn[i], got, want)
