@@ -10,6 +10,7 @@ from fractions import Fraction
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 
 def _round_f32(fr: Fraction) -> np.float32:
@@ -101,3 +102,26 @@ def test_dequantize_nested_composes(oracle_mod):
     # and it stays close to the plain dequantization
     y0 = oracle_mod.dequantize_blockwise(nf4, q, a, n, B)
     assert np.max(np.abs(y - y0)) <= np.max(np.abs(r - a)) * 1.0001
+
+
+@settings(max_examples=80, deadline=None)
+@given(nb=st.integers(1, 1500), mu=st.floats(-12, 2), sigma=st.floats(0, 3), seed=st.integers(0, 2**32 - 1))
+def test_nested_random_scales(oracle_mod, nb, mu, sigma, seed):
+    """Random counts (one block, full and ragged last blocks) and scale spreads: the offset is
+    within one binary32 ulp of the exact mean, every second-level scale is its block's largest
+    |a - offset|, and every rebuilt scale is within half the code's largest gap of the original
+    (plus the rebuild's two roundings)."""
+    code = oracle_mod.code_dynamic_signed()
+    a = np.random.default_rng(seed).lognormal(mu, sigma, nb).astype(np.float32)
+    q, a2, off = oracle_mod.nest_absmax(a, code)
+    exact = sum((Fraction(float(v)) for v in a), Fraction(0)) / nb
+    assert abs(Fraction(float(off)) - exact) <= Fraction(float(np.spacing(np.float32(float(exact)))))
+    c = a - np.float32(off)
+    want = np.array([np.max(np.abs(c[i:i + 256])) for i in range(0, nb, 256)], np.float32)
+    np.testing.assert_array_equal(a2, want)
+    r = oracle_mod.unnest_absmax(q, a2, off, code).astype(np.float64)
+    gap = np.max(np.diff(code.astype(np.float64)))
+    blk = np.repeat(a2.astype(np.float64), 256)[:nb]
+    tol = blk * gap / 2 * (1 + 1e-6) + 2 * np.spacing(np.abs(r).astype(np.float32)).astype(np.float64) \
+        + np.spacing(np.float32(abs(off))).astype(np.float64)
+    assert np.all(np.abs(r - a) <= tol)
