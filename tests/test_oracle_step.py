@@ -14,6 +14,7 @@ nearest-code requantize" against torch and an exact brute-force nearest code.
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 HP = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
 
@@ -363,3 +364,36 @@ def test_bf16_gradients_are_widened_exactly(oracle_mod):
         oracle_mod.step_tensor("adamw", p, g, m, v, None, None, None, None, 2048, step=1, **HP)
         outs.append(p)
     np.testing.assert_array_equal(outs[0], outs[1])
+
+
+_TORCH_OPT = {"adamw": "AdamW", "adam": "Adam", "momentum": "SGD", "rmsprop": "RMSprop"}
+
+
+@settings(max_examples=60, deadline=None)
+@given(optim=st.sampled_from(sorted(_TORCH_OPT)), n=st.integers(1, 600), steps=st.integers(1, 6),
+       lr=st.floats(1e-5, 1e-2), b1=st.floats(0.5, 0.99), b2=st.floats(0.9, 0.9999),
+       eps=st.sampled_from([1e-10, 1e-8, 1e-6]), wd=st.sampled_from([0.0, 1e-3, 0.1]), seed=st.integers(0, 2**31))
+def test_32bit_step_matches_torch_random_hyperparameters(oracle_mod, optim, n, steps, lr, b1, b2, eps, wd, seed):
+    """Random hyper-parameters, lengths and step counts: the 32-bit oracle step tracks
+    torch.optim (float64) for AdamW, Adam (L2), SGD with momentum and RMSprop (alpha = beta1)."""
+    p0 = (np.random.default_rng(seed).standard_normal(n) * 0.02).astype(np.float32)
+    grads = _grads(n, steps, seed + 1)
+    p = p0.copy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32) if optim in ("adamw", "adam") else None
+    for t, g in enumerate(grads, 1):
+        oracle_mod.step_tensor(optim, p, g, m, v, None, None, None, None, 256, step=t,
+                               lr=lr, beta1=b1, beta2=b2 if v is not None else 0.0, eps=eps, weight_decay=wd)
+    kw = dict(lr=_f(lr), weight_decay=_f(wd), foreach=False)
+    if optim in ("adamw", "adam"):
+        kw.update(betas=(_f(b1), _f(b2)), eps=_f(eps))
+    elif optim == "momentum":
+        kw.update(momentum=_f(b1))
+    else:
+        kw.update(alpha=_f(b1), eps=_f(eps))
+    pt, st_ = _torch_run(getattr(torch.optim, _TORCH_OPT[optim]), p0, grads, **kw)
+    _close(p, pt, np.abs(p0) + np.abs(pt - p0) + lr * steps, rtol=4e-6, ulps=8)
+    first = {"adamw": "exp_avg", "adam": "exp_avg", "momentum": "momentum_buffer", "rmsprop": "square_avg"}[optim]
+    _close(m, st_[first].numpy(), np.max(np.abs(m)), rtol=5e-5)
+    if v is not None:
+        _close(v, st_["exp_avg_sq"].numpy(), np.max(v), rtol=5e-5)
