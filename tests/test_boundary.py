@@ -282,3 +282,15 @@ def test_bench_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "params/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_gpu_check_programs_build_for_sm100a(tmp_path):
+    """The stand-alone GPU check programs under tests/gpu_checks build for sm_100a from the
+    library's own device header (compiled here, run only by the -m gpu tests)."""
+    from block_wise_bit_b200 import build as BLD
+    checks = os.path.join(ROOT, "tests", "gpu_checks")
+    for name in sorted(os.listdir(checks)):
+        if name.endswith(".cu"):
+            subprocess.run([BLD.nvcc()] + BLD.ARCH + ["-O3", "-std=c++17", "--fmad=false", "-c", "-o",
+                                                      str(tmp_path / (name + ".o")), os.path.join(checks, name)],
+                           check=True)
