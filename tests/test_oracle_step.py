@@ -397,3 +397,67 @@ def test_32bit_step_matches_torch_random_hyperparameters(oracle_mod, optim, n, s
     _close(m, st_[first].numpy(), np.max(np.abs(m)), rtol=5e-5)
     if v is not None:
         _close(v, st_["exp_avg_sq"].numpy(), np.max(v), rtol=5e-5)
+
+
+@settings(max_examples=50, deadline=None)
+@given(optim=st.sampled_from(sorted(_TORCH_OPT)), n=st.integers(1, 5000), B=st.sampled_from([256, 2048]),
+       t=st.integers(1, 30), lr=st.floats(1e-5, 1e-2), b1=st.floats(0.5, 0.99), b2=st.floats(0.9, 0.9999),
+       wd=st.sampled_from([0.0, 0.01]), seed=st.integers(0, 2**31))
+def test_8bit_step_random_state_matches_torch(oracle_mod, optim, n, B, t, lr, b1, b2, wd, seed):
+    """Random 8-bit states, scales, hyper-parameters and lengths: the step equals torch.optim run
+    from the dequantized state, each new block scale is the block's largest new |state|, and
+    each new code is the exact nearest code of state / scale wherever that quotient is not
+    within a relative 1e-5 of a decision midpoint."""
+    rng = np.random.default_rng(seed)
+    two = optim in ("adamw", "adam")
+    c1 = oracle_mod.code_dynamic_unsigned() if optim == "rmsprop" else oracle_mod.code_dynamic_signed()
+    c2 = oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    q1 = rng.integers(0, 256, n).astype(np.uint8)
+    q2 = rng.integers(0, 256, n).astype(np.uint8)
+    a1 = rng.uniform(1e-8, 1e-6, nb).astype(np.float32) if optim == "rmsprop" else \
+        rng.uniform(1e-4, 1e-3, nb).astype(np.float32)
+    a2 = rng.uniform(1e-8, 1e-6, nb).astype(np.float32)
+    m0 = (c1[q1] * np.repeat(a1, B)[:n]).astype(np.float32)  # the dequantized state, binary32
+    v0 = (c2[q2] * np.repeat(a2, B)[:n]).astype(np.float32)
+    p = p0.copy()
+    oracle_mod.step_tensor(optim, p, g, q1, q2 if two else None, a1, a2 if two else None, c1, c2 if two else None,
+                           B, step=t, lr=lr, beta1=b1, beta2=b2 if two else 0.0, eps=1e-8, weight_decay=wd)
+
+    tp = torch.nn.Parameter(torch.from_numpy(p0.astype(np.float64)))
+    kw = dict(lr=_f(lr), weight_decay=_f(wd), foreach=False)
+    m64 = torch.from_numpy(m0.astype(np.float64))
+    if two:
+        kw.update(betas=(_f(b1), _f(b2)), eps=_f(1e-8))
+        state = {"step": torch.tensor(float(t - 1)), "exp_avg": m64, "exp_avg_sq": torch.from_numpy(v0.astype(np.float64))}
+    elif optim == "momentum":
+        kw.update(momentum=_f(b1))
+        state = {"momentum_buffer": m64}
+    else:
+        kw.update(alpha=_f(b1), eps=_f(1e-8))
+        state = {"step": torch.tensor(float(t - 1)), "square_avg": m64}
+    opt = getattr(torch.optim, _TORCH_OPT[optim])([tp], **kw)
+    opt.state[tp] = state
+    tp.grad = torch.from_numpy(g.astype(np.float64))
+    opt.step()
+    pt = tp.detach().numpy()
+    _close(p, pt, np.abs(p0) + np.abs(pt - p0) + lr, rtol=4e-6, ulps=8)
+
+    first = {"adamw": "exp_avg", "adam": "exp_avg", "momentum": "momentum_buffer", "rmsprop": "square_avg"}[optim]
+    checks = [(a1, q1, opt.state[tp][first].numpy(), c1)]
+    if two:
+        checks.append((a2, q2, opt.state[tp]["exp_avg_sq"].numpy(), c2))
+    for a, q, s, code in checks:
+        want_a = np.array([np.max(np.abs(s[i:i + B])) for i in range(0, n, B)])
+        np.testing.assert_allclose(a, want_a, rtol=2e-5)
+        xn = s / np.repeat(want_a, B)[:n]
+        mids = (code[:-1].astype(np.float64) + code[1:].astype(np.float64)) / 2
+        k = np.clip(np.searchsorted(mids, xn), 1, mids.size - 1)
+        gap = np.minimum(np.abs(xn - mids[k - 1]), np.abs(xn - mids[np.minimum(k, mids.size - 1)]))
+        far = gap > 1e-5 * np.maximum(np.abs(xn), 1e-7)
+        qq, _ = _nearest_exact(code, xn)
+        np.testing.assert_array_equal(q[far], qq[far])
+        if n >= 1000:
+            assert far.mean() > 0.95
