@@ -294,3 +294,23 @@ def test_gpu_check_programs_build_for_sm100a(tmp_path):
             subprocess.run([BLD.nvcc()] + BLD.ARCH + ["-O3", "-std=c++17", "--fmad=false", "-c", "-o",
                                                       str(tmp_path / (name + ".o")), os.path.join(checks, name)],
                            check=True)
+
+
+def test_host_tensors_are_refused_without_fallback():
+    """The compute wrappers take CUDA tensors only: host tensors are refused in Python before the
+    library is called (there is no CPU path to fall back to), for the standalone calls and the
+    optimizer front end alike."""
+    import torch
+    from block_wise_bit_b200 import optim as O
+    code = B.bnbq_codebook("dynamic_signed")
+    x = torch.zeros(4096)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        B.bnbq_quantize_blockwise(code, x, 2048, absmax=torch.zeros(2), out=torch.zeros(4096, dtype=torch.uint8))
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        B.bnbq_dequantize_blockwise(code, torch.zeros(4096, dtype=torch.uint8), torch.ones(2), 2048,
+                                    out=torch.zeros(4096))
+    p = torch.nn.Parameter(torch.zeros(8192))
+    p.grad = torch.zeros(8192)
+    with pytest.raises((TypeError, RuntimeError, AssertionError)):
+        O.AdamW8bit([p], lr=1e-3).step()
+    assert torch.equal(p.detach(), torch.zeros(8192))
