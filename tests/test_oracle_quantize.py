@@ -322,7 +322,8 @@ def test_quantize_random_blocks_match_bruteforce(oracle_mod, x, B, name):
     """Random lengths (empty and ragged included), blocksizes, codebooks and values (zeros,
     subnormals, huge values, exact codes): each block's scale is its largest magnitude and each
     element takes the exact nearest code of its binary32 quotient (ties and rounded midpoints to
-    the lower code), packed two per byte for 4-bit codes."""
+    the lower code), packed two per byte for 4-bit codes; dequantizing gives code * scale in
+    binary32 within half a code gap of x, and bf16 output is that value rounded as torch does."""
     code = _codes(oracle_mod)[name]
     xs = np.array(x, np.float32)
     if code.min() >= 0:
@@ -346,3 +347,12 @@ def test_quantize_random_blocks_match_bruteforce(oracle_mod, x, B, name):
             want = _argmin_exact(code, xn[i])
             got = int(qi[s + i])
             assert got == want or (_is_rounded_mid(code, xn[i]) and got == want - 1), (b, i, xn[i], got, want)
+    # dequantize: within half the code's largest gap of x (times the block scale), and the bf16
+    # output is torch's rounding of the fp32 output
+    y = oracle_mod.dequantize_blockwise(code, q, absmax, n, B)
+    np.testing.assert_array_equal(y, (code[qi] * np.repeat(absmax, B)[:n]).astype(np.float32))
+    gap = np.max(np.diff(code.astype(np.float64)))
+    scale = np.repeat(absmax.astype(np.float64), B)[:n]
+    assert np.all(np.abs(y.astype(np.float64) - xs) <= scale * gap / 2 * (1 + 1e-6) + np.spacing(np.abs(y)))
+    yb = oracle_mod.dequantize_blockwise(code, q, absmax, n, B, out_bf16=True)
+    np.testing.assert_array_equal(yb, torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
