@@ -126,11 +126,17 @@ def _dtype_id(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
 
 
-def _dev(t: torch.Tensor, name: str) -> int:
+def _dev(t: torch.Tensor, name: str, device: Optional[int] = None) -> int:
+    """Device pointer of ``t``, which must be a contiguous CUDA tensor on the current device (the
+    library launches on the current device; ``device`` passes it in when already known)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    cur = torch.cuda.current_device() if device is None else device
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{cur}; "
+                         f"call inside torch.cuda.device({t.device.index})")
     return t.data_ptr()
 
 
@@ -246,16 +252,19 @@ class TensorState:
 
 def pack_tensor_list(tensors: Sequence[TensorState]):
     arr = (CTensor * max(1, len(tensors)))()
+    cur = None  # the current device, looked up once the first tensor is known to be on CUDA
     for i, t in enumerate(tensors):
         if t.p.dtype != torch.float32:
             raise TypeError("parameters must be float32")
         c = arr[i]
-        c.p = _dev(t.p, "p")
-        c.g = _dev(t.g, "g")
-        c.state1 = _dev(t.state1, "state1")
-        c.state2 = _dev(t.state2, "state2") if t.state2 is not None else None
-        c.absmax1 = _dev(t.absmax1, "absmax1") if t.absmax1 is not None else None
-        c.absmax2 = _dev(t.absmax2, "absmax2") if t.absmax2 is not None else None
+        c.p = _dev(t.p, "p", cur)
+        if cur is None:
+            cur = t.p.device.index
+        c.g = _dev(t.g, "g", cur)
+        c.state1 = _dev(t.state1, "state1", cur)
+        c.state2 = _dev(t.state2, "state2", cur) if t.state2 is not None else None
+        c.absmax1 = _dev(t.absmax1, "absmax1", cur) if t.absmax1 is not None else None
+        c.absmax2 = _dev(t.absmax2, "absmax2", cur) if t.absmax2 is not None else None
         c.n = t.p.numel()
         c.g_dtype = _dtype_id(t.g)
         c.state_bits = t.state_bits

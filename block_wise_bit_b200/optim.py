@@ -12,6 +12,7 @@ list; each ``step()`` is one call of the CUDA library per parameter group.
 """
 from __future__ import annotations
 
+import contextlib
 from typing import Dict, List, Optional
 
 import torch
@@ -68,7 +69,6 @@ class Optimizer8bit(torch.optim.Optimizer):
         self.blocksize = blocksize
         self.optim_bits = optim_bits
         self._force32: set = set()
-        self._packed: Dict[int, tuple] = {}
 
     @property
     def two_states(self) -> bool:
@@ -94,14 +94,18 @@ class Optimizer8bit(torch.optim.Optimizer):
         if closure is not None:
             with torch.enable_grad():
                 loss = closure()
-        for gi, group in enumerate(self.param_groups):
+        for group in self.param_groups:
             params = [p for p in group["params"] if p.grad is not None]
             if not params:
                 continue
             dev = params[0].device
+            if any(p.device != dev for p in params):
+                raise ValueError("the parameters of one group must be on one device")
             code1 = device_codebook(self.code1_kind, dev)
             code2 = device_codebook("dynamic_unsigned", dev) if self.two_states else None
-            entries: List[B.TensorState] = []
+            # Each parameter keeps its own step count, as in torch.optim (a parameter whose first
+            # gradient comes later starts its bias correction at 1); one call per distinct count.
+            by_step: Dict[int, List[B.TensorState]] = {}
             for p in params:
                 if p.dtype != torch.float32 or not p.is_contiguous():
                     raise TypeError("8-bit optimizers here step contiguous float32 parameters")
@@ -111,13 +115,15 @@ class Optimizer8bit(torch.optim.Optimizer):
                     st["step"] = 0
                 st["step"] += 1
                 g = p.grad if p.grad.is_contiguous() else p.grad.contiguous()
-                entries.append(B.TensorState(p.view(-1), g.view(-1), st["state1"], st.get("state2"),
-                                             st.get("absmax1"), st.get("absmax2")))
-            t = self.state[params[0]]["step"]
+                by_step.setdefault(st["step"], []).append(
+                    B.TensorState(p.view(-1), g.view(-1), st["state1"], st.get("state2"), st.get("absmax1"),
+                                  st.get("absmax2")))
             b1, b2 = group["betas"]
-            B.bnbq_step_8bit(self._KIND, entries, lr=group["lr"], beta1=b1, beta2=b2, eps=group["eps"],
-                             weight_decay=group["weight_decay"], step=t, code1=code1, code2=code2,
-                             blocksize=self.blocksize)
+            with torch.cuda.device(dev) if dev.type == "cuda" else contextlib.nullcontext():
+                for t, entries in by_step.items():
+                    B.bnbq_step_8bit(self._KIND, entries, lr=group["lr"], beta1=b1, beta2=b2, eps=group["eps"],
+                                     weight_decay=group["weight_decay"], step=t, code1=code1, code2=code2,
+                                     blocksize=self.blocksize)
         return loss
 
 

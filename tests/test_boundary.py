@@ -314,3 +314,36 @@ def test_host_tensors_are_refused_without_fallback():
     with pytest.raises((TypeError, RuntimeError, AssertionError)):
         O.AdamW8bit([p], lr=1e-3).step()
     assert torch.equal(p.detach(), torch.zeros(8192))
+
+
+def test_front_end_keeps_a_step_count_per_parameter(monkeypatch):
+    """As in torch.optim, each parameter counts its own steps: a parameter whose first gradient
+    arrives later starts its bias correction at step 1, so the front end makes one library call
+    per distinct count (recorded here in place of the CUDA call)."""
+    import torch
+    from block_wise_bit_b200 import optim as O
+    calls = []
+    monkeypatch.setattr(O.B, "bnbq_step_8bit",
+                        lambda kind, entries, step, **kw: calls.append((kind, step, [e.p.numel() for e in entries])))
+    p1, p2 = torch.nn.Parameter(torch.zeros(5000)), torch.nn.Parameter(torch.zeros(6000))
+    opt = O.AdamW8bit([p1, p2], lr=1e-3)
+    p1.grad = torch.ones(5000)
+    opt.step()
+    p2.grad = torch.ones(6000)
+    opt.step()
+    opt.step()
+    assert calls == [("adamw", 1, [5000]), ("adamw", 2, [5000]), ("adamw", 1, [6000]),
+                     ("adamw", 3, [5000]), ("adamw", 2, [6000])]
+    assert opt.state[p1]["step"] == 3 and opt.state[p2]["step"] == 2
+
+
+def test_front_end_refuses_a_group_on_several_devices(monkeypatch):
+    import torch
+    from block_wise_bit_b200 import optim as O
+    monkeypatch.setattr(O.B, "bnbq_step_8bit", lambda *a, **kw: pytest.fail("must not be called"))
+    p1 = torch.nn.Parameter(torch.zeros(5000))
+    p2 = torch.nn.Parameter(torch.zeros(5000, device="meta"))
+    p1.grad = torch.ones(5000)
+    p2.grad = torch.ones(5000, device="meta")
+    with pytest.raises(ValueError, match="one device"):
+        O.AdamW8bit([p1, p2], lr=1e-3).step()
