@@ -461,3 +461,32 @@ def test_8bit_step_random_state_matches_torch(oracle_mod, optim, n, B, t, lr, b1
         np.testing.assert_array_equal(q[far], qq[far])
         if n >= 1000:
             assert far.mean() > 0.95
+
+
+@settings(max_examples=60, deadline=None)
+@given(optim=st.sampled_from(["adamw", "adam", "lion", "momentum", "rmsprop"]), n=st.integers(1, 9000),
+       B=st.sampled_from([256, 2048]), split=st.floats(0, 1), t=st.integers(1, 9), seed=st.integers(0, 2**31))
+def test_blocks_are_independent(oracle_mod, optim, n, B, split, t, seed):
+    """Blocks are quantized and stepped independently (abstract of "8-bit Optimizers via
+    Block-wise Quantization"): stepping the block range in two parts, at any split, gives exactly
+    the result of one call over all blocks."""
+    rng = np.random.default_rng(seed)
+    two = optim in ("adamw", "adam")
+    c1 = oracle_mod.code_dynamic_unsigned() if optim == "rmsprop" else oracle_mod.code_dynamic_signed()
+    c2 = oracle_mod.code_dynamic_unsigned()
+    nb = (n + B - 1) // B
+    k = int(round(split * nb))
+    base = dict(p=(rng.standard_normal(n) * 0.02).astype(np.float32),
+                g=(rng.standard_normal(n) * 1e-3).astype(np.float32),
+                q1=rng.integers(0, 256, n).astype(np.uint8), q2=rng.integers(0, 256, n).astype(np.uint8),
+                a1=rng.uniform(1e-8, 1e-3, nb).astype(np.float32), a2=rng.uniform(1e-8, 1e-6, nb).astype(np.float32))
+    hp = dict(lr=1e-3, beta1=0.9, beta2=0.999 if two else 0.0, eps=1e-8, weight_decay=0.01)
+    runs = []
+    for ranges in ([(0, nb)], [(0, k), (k, nb)]):
+        d = {key: v.copy() for key, v in base.items()}
+        for r in ranges:
+            oracle_mod.step_tensor(optim, d["p"], d["g"], d["q1"], d["q2"] if two else None, d["a1"],
+                                   d["a2"] if two else None, c1, c2 if two else None, B, step=t, block_range=r, **hp)
+        runs.append(d)
+    for key in base:
+        np.testing.assert_array_equal(runs[0][key], runs[1][key])
