@@ -135,6 +135,94 @@ def bench_quant(args, base):
                peak_gbs=peak, gpu_launches=(5 if nested else 2) * args.steps)
     print(json.dumps(out))
 
+def bench_zero1(args, base, shape, optim, seed, hp, outlier):
+    """ZeRO-1 data-parallel step over the whole list on ``world`` ranks: every rank holds the full
+    flat parameters and its own full bf16 gradient; per step the gradients are reduce-scattered in
+    place, each rank steps its block-aligned share (optimizer state exists only for it), and the
+    parameters are all-gathered in place.  ``value``: parameters of the list stepped per second
+    (the list is stepped once per step by all ranks together: strong scaling), with the two
+    collectives and the step kernel timed separately (CUDA events, slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    import block_wise_bit_b200 as bq
+    from block_wise_bit_b200 import optim as O
+    from block_wise_bit_b200 import workloads as W
+    from block_wise_bit_b200 import zero
+    from datetime import timedelta
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if "MASTER_ADDR" not in os.environ:  # one process without a launcher
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(29500 + os.getpid() % 1000))
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=120),
+                            device_id=dev)
+    B = 2048
+    lay = W.Layout.build(W.SHAPES[shape](), B)
+    numels = [sp.numel for sp in lay.specs]
+    ex = zero.ZeroOneExchange(numels, B, world, rank)
+    P = torch.zeros(ex.total, device=dev)
+    G = torch.zeros(ex.total, device=dev, dtype=torch.bfloat16)
+    for i, spec in enumerate(lay.specs):
+        ex.views(P, i).copy_(W.normal(spec.numel, 0.02, dev, shape, seed, i, "p"))
+        W.grad_fill_(ex.views(G, i), 1e-3, outlier[0], outlier[1], shape, seed, rank, i, "g")
+    two = optim in ("adamw", "adam")
+    code1 = O.device_codebook("dynamic_unsigned" if optim == "rmsprop" else "dynamic_signed", dev)
+    code2 = O.device_codebook("dynamic_unsigned", dev) if two else None
+    entries = []
+    for pc, pv, gv in ex.piece_views(P, G):
+        st = O.new_state(pv, two, lay.state_bits[pc.tensor], B, code1, code2)
+        entries.append(bq.TensorState(pv, gv, st["state1"], st.get("state2"), st.get("absmax1"), st.get("absmax2")))
+    packed = bq.pack_tensor_list(entries)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(t, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ex.reduce_scatter_grads(G)
+        if ev is not None:
+            ev[1].record(stream)
+        if entries:
+            bq.bnbq_step_8bit(optim, packed, ntensors=len(entries), step=t, code1=code1, code2=code2, blocksize=B,
+                              **hp)
+        if ev is not None:
+            ev[2].record(stream)
+        ex.all_gather_params(P)
+        if ev is not None:
+            ev[3].record(stream)
+
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        one_step(t)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        t += 1
+        one_step(t, evs[k])
+    torch.cuda.synchronize()
+    dist.barrier()
+    parts = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(3)]
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    total_ms = max_over_ranks(total_ms, dev, world)
+    parts = [max_over_ranks(x, dev, world) for x in parts]
+    flags = bq.bnbq_device_flags(clear=True)
+    if rank == 0:
+        cfg = dict(base["config"], workload=f"{args.workload}8bit_zero1", parallelism=f"zero1 x{world}",
+                   rank_share_params=sum(pc.numel for pc in ex.pieces[0]))
+        out = dict(base, config=cfg, scaling="strong", value=lay.n_params * args.steps / (total_ms / 1e3),
+                   n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=round(total_ms / args.steps, 4),
+                   zero1={"reduce_scatter_ms": round(parts[0], 4), "step_ms": round(parts[1], 4),
+                          "all_gather_ms": round(parts[2], 4), "grad_bytes": 2 * ex.total, "param_bytes": 4 * ex.total},
+                   cpu_baseline=None, e2e=None, gpu_launches=args.steps, device_flags=flags)
+        print(json.dumps(out))
+    dist.destroy_process_group()
+
+
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "block_wise_bit_b200", "csrc", f) for f in
                   ("bnbq_step.cu", "bnbq_device.cuh", "bnbq_internal.h")]
@@ -356,6 +444,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--zero1", action="store_true",
+                    help="ZeRO-1 data-parallel step: reduce-scatter of gradients, each rank steps its share, "
+                         "all-gather of parameters (NCCL)")
     ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="8-bit elements in the CPU oracle sample")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="wall time the CPU baseline aims for (consecutive oracle steps over the sample)")
@@ -411,6 +502,8 @@ def main():
 
     if args.workload.startswith("quant"):
         return bench_quant(args, base)
+    if args.zero1:
+        return bench_zero1(args, base, shape, optim, seed, hp, (ofrac, oscale))
 
     if world > 1:
         from datetime import timedelta

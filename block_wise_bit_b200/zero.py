@@ -2,11 +2,10 @@
 
 Blocks are independent (abstract of "8-bit Optimizers via Block-wise Quantization": each block is
 quantized on its own and processed in parallel), so the optimizer step shards without any
-exchange: split the list's blocks -- numbered tensor by tensor -- into contiguous ranges of
-near-equal element count, and let each rank step its range.  A range may cut a tensor, but only
-between two of its blocks, so every block (and its absmax) belongs to exactly one rank.
-Collectives before and after the step (reduce-scatter of gradients, all-gather of parameters) are
-outside the step and outside this module.
+exchange: each rank steps one contiguous range of the list's blocks.  A range may cut a tensor,
+but only between two of its blocks, so every block (and its absmax) belongs to exactly one rank.
+The collectives of a data-parallel step -- reduce-scatter of gradients before the step,
+all-gather of parameters after it -- are outside the step kernel (``ZeroOneExchange``).
 """
 from __future__ import annotations
 
@@ -78,68 +77,79 @@ def shard_states(states: Sequence[B.TensorState], pieces: Sequence[Piece], block
 class ZeroOneExchange:
     """The collectives of a ZeRO-1 step over one flat parameter list, around the unchanged step.
 
-    Every rank holds the whole flat parameter buffer and its own full gradient (data parallel);
-    rank r owns the pieces ``partition(...)[r]``, i.e. one contiguous, block-aligned range of the
-    flat buffer (tensors sit at ``offsets`` in it, in list order).  One step is:
+    Flat layout: tensor i occupies ``[offsets[i], offsets[i] + numels[i])`` of a flat buffer whose
+    offsets are multiples of the blocksize, so every offset that is a multiple of the blocksize is
+    a block boundary of whatever tensor it falls in.  The buffer is ``world * chunk`` elements
+    long (``chunk`` a multiple of the blocksize, the tail is padding) and rank r owns
+    ``[r * chunk, (r + 1) * chunk)``: an equal, block-aligned share.  Every rank holds the whole
+    flat parameter buffer and its own full gradient (data parallel).  One step is:
 
-      1. ``reduce_scatter_grads``: the gradients are summed over ranks, each rank receiving only
-         its own range (ranges are padded to one common chunk length so that the equal-size
-         ``reduce_scatter`` collective applies);
-      2. the rank steps its pieces with the summed gradient (``piece_views`` gives the slices;
-         the optimizer state exists only for the rank's pieces);
-      3. ``all_gather_params``: every rank's stepped range is gathered back into every rank's
-         flat parameter buffer.
+      1. ``reduce_scatter_grads``: the gradients are summed over ranks into this rank's range of
+         its own gradient buffer, in place (``reduce_scatter_tensor`` on the flat buffer);
+      2. the rank steps its pieces with the summed gradient (``piece_views``; the optimizer state
+         exists only for the rank's pieces);
+      3. ``all_gather_params``: every rank's stepped range is gathered into every rank's flat
+         parameter buffer, in place (``all_gather_into_tensor``).
 
-    Works with any torch.distributed backend that has ``reduce_scatter`` and
-    ``all_gather_into_tensor`` (NCCL on GPUs, gloo on CPU).  A multi-GPU run is not part of this
-    repository's tests (they have one GPU); the exchange is checked with gloo ranks on CPU.
+    No staging copies: both collectives read and write the flat buffers directly.  Works with any
+    torch.distributed backend that has ``reduce_scatter_tensor`` and ``all_gather_into_tensor``
+    (NCCL on GPUs, gloo on CPU).
     """
 
-    def __init__(self, numels: Sequence[int], offsets: Sequence[int], blocksize: int, world: int, rank: int,
-                 align: int = 16):
+    def __init__(self, numels: Sequence[int], blocksize: int, world: int, rank: int):
+        if world < 1 or not 0 <= rank < world:
+            raise ValueError("need 0 <= rank < world")
         self.world, self.rank, self.blocksize = world, rank, blocksize
-        self.numels, self.offsets = list(numels), list(offsets)
-        self.pieces = partition(numels, blocksize, world)
-        self.ranges = []
-        for pcs in self.pieces:
-            if pcs:
-                lo = self.offsets[pcs[0].tensor] + pcs[0].start
-                hi = self.offsets[pcs[-1].tensor] + pcs[-1].start + pcs[-1].numel
-            else:
-                lo = hi = 0
-            self.ranges.append((lo, hi))
-        longest = max(hi - lo for lo, hi in self.ranges)
-        self.chunk = max(align, (longest + align - 1) // align * align)
+        self.numels = list(numels)
+        self.offsets, o = [], 0
+        for n in self.numels:
+            self.offsets.append(o)
+            o += (n + blocksize - 1) // blocksize * blocksize
+        blocks = o // blocksize
+        self.chunk = max(1, (blocks + world - 1) // world) * blocksize
+        self.total = world * self.chunk
+        self.pieces = [self._pieces(r) for r in range(world)]
 
-    def reduce_scatter_grads(self, g_flat, group=None):
-        """Sum of every rank's gradient over this rank's range (a tensor of ``chunk`` elements;
-        the first ``hi - lo`` are meaningful)."""
-        import torch
-        import torch.distributed as dist
-        staged = torch.zeros(self.world * self.chunk, dtype=g_flat.dtype, device=g_flat.device)
-        for r, (lo, hi) in enumerate(self.ranges):
-            staged[r * self.chunk:r * self.chunk + hi - lo].copy_(g_flat[lo:hi])
-        out = torch.empty(self.chunk, dtype=g_flat.dtype, device=g_flat.device)
-        dist.reduce_scatter(out, list(staged.split(self.chunk)), group=group)
+    @property
+    def range(self):
+        """This rank's range of the flat buffers."""
+        return self.rank * self.chunk, (self.rank + 1) * self.chunk
+
+    def _pieces(self, r: int) -> List[Piece]:
+        lo, hi = r * self.chunk, (r + 1) * self.chunk
+        out = []
+        for t, (n, off) in enumerate(zip(self.numels, self.offsets)):
+            a, b = max(lo, off), min(hi, off + n)
+            if a >= b:
+                continue
+            s, e = a - off, b - off  # s is a multiple of the blocksize (block boundary)
+            nb = (e - s + self.blocksize - 1) // self.blocksize
+            out.append(Piece(t, s // self.blocksize, nb, s, e - s))
         return out
 
-    def piece_views(self, p_flat, g_chunk):
-        """(piece, parameter slice, summed-gradient slice) for each of this rank's pieces."""
-        lo = self.ranges[self.rank][0]
+    def views(self, flat, t: int):
+        """Tensor t's slice of a flat buffer."""
+        return flat[self.offsets[t]:self.offsets[t] + self.numels[t]]
+
+    def reduce_scatter_grads(self, g_flat, group=None):
+        """Sum every rank's gradient over this rank's range, written into ``g_flat`` in place;
+        returns that range (a view)."""
+        import torch.distributed as dist
+        lo, hi = self.range
+        out = g_flat[lo:hi]
+        dist.reduce_scatter_tensor(out, g_flat[:self.total], group=group)
+        return out
+
+    def piece_views(self, p_flat, g_flat):
+        """(piece, parameter slice, gradient slice) for each of this rank's pieces."""
         out = []
         for pc in self.pieces[self.rank]:
             a = self.offsets[pc.tensor] + pc.start
-            out.append((pc, p_flat[a:a + pc.numel], g_chunk[a - lo:a - lo + pc.numel]))
+            out.append((pc, p_flat[a:a + pc.numel], g_flat[a:a + pc.numel]))
         return out
 
     def all_gather_params(self, p_flat, group=None):
-        """Copy every rank's range of the flat parameters from that rank into ``p_flat``."""
-        import torch
+        """Every rank's range of the flat parameters, from that rank into ``p_flat``, in place."""
         import torch.distributed as dist
-        lo, hi = self.ranges[self.rank]
-        mine = torch.zeros(self.chunk, dtype=p_flat.dtype, device=p_flat.device)
-        mine[:hi - lo].copy_(p_flat[lo:hi])
-        gathered = torch.empty(self.world * self.chunk, dtype=p_flat.dtype, device=p_flat.device)
-        dist.all_gather_into_tensor(gathered, mine, group=group)
-        for r, (a, b) in enumerate(self.ranges):
-            p_flat[a:b].copy_(gathered[r * self.chunk:r * self.chunk + b - a])
+        lo, hi = self.range
+        dist.all_gather_into_tensor(p_flat[:self.total], p_flat[lo:hi], group=group)

@@ -139,26 +139,15 @@ def test_two_gloo_ranks_reproduce_single_rank_step(oracle_mod):
 
 
 # ------------------------------------------------------------------ the ZeRO-1 exchange, 2 gloo ranks
-OFFS_ALIGN = 16
-
-
-def _flat_offsets(numels):
-    offs, o = [], 0
-    for n in numels:
-        offs.append(o)
-        o += (n + OFFS_ALIGN - 1) // OFFS_ALIGN * OFFS_ALIGN  # gaps between tensors, as in the flat layouts
-    return offs, o
-
-
 def _exchange_inputs(world):
     rng = np.random.default_rng(7)
-    offs, total = _flat_offsets(NUMELS)
-    p = np.zeros(total, np.float32)
-    for n, o in zip(NUMELS, offs):
+    ex = zero.ZeroOneExchange(NUMELS, B, world, 0)
+    p = np.zeros(ex.total, np.float32)
+    for n, o in zip(NUMELS, ex.offsets):
         p[o:o + n] = (rng.standard_normal(n) * 0.02).astype(np.float32)
-    grads = [np.zeros(total, np.float32) for _ in range(world)]
+    grads = [np.zeros(ex.total, np.float32) for _ in range(world)]
     for r in range(world):
-        for n, o in zip(NUMELS, offs):
+        for n, o in zip(NUMELS, ex.offsets):
             grads[r][o:o + n] = (rng.standard_normal(n) * 1e-3).astype(np.float32)
     states = []
     for n in NUMELS:
@@ -166,7 +155,7 @@ def _exchange_inputs(world):
         states.append(dict(s1=rng.integers(0, 256, n).astype(np.uint8), s2=rng.integers(0, 256, n).astype(np.uint8),
                            a1=rng.uniform(1e-4, 1e-3, nb).astype(np.float32),
                            a2=rng.uniform(1e-8, 1e-6, nb).astype(np.float32)))
-    return offs, p, grads, states
+    return ex.offsets, p, grads, states
 
 
 def _exchange_worker(rank, world, port, q):
@@ -177,11 +166,11 @@ def _exchange_worker(rank, world, port, q):
         import oracle
         offs, p, grads, states = _exchange_inputs(world)
         c1, c2 = oracle.code_dynamic_signed(), oracle.code_dynamic_unsigned()
-        ex = zero.ZeroOneExchange(NUMELS, offs, B, world, rank)
-        P = torch.from_numpy(p)
-        g_chunk = ex.reduce_scatter_grads(torch.from_numpy(grads[rank]))
+        ex = zero.ZeroOneExchange(NUMELS, B, world, rank)
+        P, G = torch.from_numpy(p), torch.from_numpy(grads[rank])
+        ex.reduce_scatter_grads(G)
         mine = []
-        for pc, pv, gv in ex.piece_views(P, g_chunk):
+        for pc, pv, gv in ex.piece_views(P, G):
             st = states[pc.tensor]
             b0, b1 = pc.first_block, pc.first_block + pc.n_blocks
             s = {k: np.ascontiguousarray(st[k][pc.start:pc.start + pc.numel]) for k in ("s1", "s2")}
@@ -198,8 +187,9 @@ def _exchange_worker(rank, world, port, q):
 
 def test_zero1_exchange_two_gloo_ranks_equals_single_rank_step(oracle_mod):
     """Reduce-scatter of the gradients, a step of each rank's pieces, all-gather of the
-    parameters: every rank ends with the parameters of one single-rank step on the summed
-    gradient, and the pieces' states equal the single-rank states, bit for bit."""
+    parameters, both collectives in place on the flat buffers: every rank ends with the
+    parameters of one single-rank step on the summed gradient, and the pieces' states equal the
+    single-rank states, bit for bit."""
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -231,43 +221,39 @@ def test_zero1_exchange_two_gloo_ranks_equals_single_rank_step(oracle_mod):
     assert covered == sum(NUMELS)
 
 
-def test_zero1_exchange_ranges():
-    """Each rank's range is contiguous, block-aligned within its tensors, ordered and disjoint;
-    together they cover every tensor; the common chunk holds the longest."""
-    offs, total = _flat_offsets(NUMELS)
+def _check_exchange_layout(numels, bs, world):
+    ex = zero.ZeroOneExchange(numels, bs, world, 0)
+    assert ex.chunk % bs == 0 and ex.total == world * ex.chunk
+    for t, (n, o) in enumerate(zip(numels, ex.offsets)):
+        assert o % bs == 0 and o + n <= ex.total
+        if t + 1 < len(numels):
+            assert ex.offsets[t + 1] >= o + n
+    owner = {}
+    for r, pcs in enumerate(ex.pieces):
+        assert pcs == zero.ZeroOneExchange(numels, bs, world, r).pieces[r]
+        for pc in pcs:
+            a = ex.offsets[pc.tensor] + pc.start
+            assert r * ex.chunk <= a and a + pc.numel <= (r + 1) * ex.chunk  # inside the rank's range
+            assert pc.start == pc.first_block * bs and pc.n_blocks >= 1
+            assert pc.numel == min(numels[pc.tensor], (pc.first_block + pc.n_blocks) * bs) - pc.start
+            owner.setdefault(pc.tensor, []).append((pc.start, pc.start + pc.numel))
+    for t, n in enumerate(numels):  # every element of every tensor on exactly one rank
+        spans = sorted(owner.get(t, []))
+        assert sum(e - s for s, e in spans) == n
+        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:])) and (not spans or spans[0][0] == 0)
+    padded = sum((n + bs - 1) // bs * bs for n in numels)
+    assert ex.chunk <= max(bs, (padded // bs + world - 1) // world * bs)  # an equal share, to one block
+
+
+def test_zero1_exchange_layout():
+    """Tensor offsets on block boundaries, equal block-aligned chunks per rank, each rank's pieces
+    inside its chunk, every element owned once."""
     for world in (1, 2, 3, 8):
-        ranges = [zero.ZeroOneExchange(NUMELS, offs, B, world, r).ranges[r] for r in range(world)]
-        ex = zero.ZeroOneExchange(NUMELS, offs, B, world, 0)
-        assert ranges == ex.ranges
-        nonempty = [(lo, hi) for lo, hi in ranges if hi > lo]
-        assert all(a[1] <= b[0] for a, b in zip(nonempty, nonempty[1:]))
-        assert nonempty[0][0] == 0 and nonempty[-1][1] == offs[-1] + NUMELS[-1]
-        assert ex.chunk >= max(hi - lo for lo, hi in ranges) and ex.chunk % 16 == 0
-        for r, pcs in enumerate(ex.pieces):
-            for pc in pcs:
-                a = offs[pc.tensor] + pc.start
-                assert ranges[r][0] <= a and a + pc.numel <= ranges[r][1]
+        _check_exchange_layout(NUMELS, B, world)
 
 
 @settings(max_examples=200, deadline=None)
 @given(numels=st.lists(st.integers(0, 20000), min_size=1, max_size=10), bs=st.sampled_from([256, 2048]),
        world=st.integers(1, 8))
-def test_zero1_exchange_ranges_on_random_lists(numels, bs, world):
-    """Random lists: the ranks' flat ranges are ordered and disjoint, each holds exactly its own
-    pieces, every element of every tensor falls in some rank's range, and the common chunk holds
-    the longest range (so the padded reduce-scatter and all-gather move every element once)."""
-    offs, _ = _flat_offsets(numels)
-    ex = zero.ZeroOneExchange(numels, offs, bs, world, 0)
-    nonempty = [(lo, hi) for lo, hi in ex.ranges if hi > lo]
-    assert all(a[1] <= b[0] for a, b in zip(nonempty, nonempty[1:]))
-    assert ex.chunk % 16 == 0 and ex.chunk >= max([hi - lo for lo, hi in ex.ranges] + [1])
-    owner = {}
-    for r, pcs in enumerate(ex.pieces):
-        for pc in pcs:
-            a = offs[pc.tensor] + pc.start
-            assert ex.ranges[r][0] <= a and a + pc.numel <= ex.ranges[r][1]
-            owner.setdefault(pc.tensor, []).append((pc.start, pc.start + pc.numel))
-    for t, n in enumerate(numels):
-        spans = sorted(owner.get(t, []))
-        assert sum(e - s for s, e in spans) == n
-        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:])) and (not spans or spans[0][0] == 0)
+def test_zero1_exchange_layout_on_random_lists(numels, bs, world):
+    _check_exchange_layout(numels, bs, world)
