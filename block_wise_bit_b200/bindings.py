@@ -140,6 +140,18 @@ def _dev(t: torch.Tensor, name: str, device: Optional[int] = None) -> int:
     return t.data_ptr()
 
 
+def _step_code(code: Optional[torch.Tensor], name: str, device: Optional[int]) -> Optional[int]:
+    """Device pointer of a step codebook: None stays None; otherwise a contiguous float32 CUDA
+    tensor of exactly 256 values on the current device (the kernel reads 256 codes)."""
+    if code is None:
+        return None
+    if not isinstance(code, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if code.dtype != torch.float32 or code.numel() != 256:
+        raise ValueError(f"{name} must hold 256 float32 codes (got {code.numel()} values of {code.dtype})")
+    return _dev(code, name, device)
+
+
 # ------------------------------------------------------------------------------------ codebooks
 def bnbq_codebook(kind: str | int) -> torch.Tensor:
     """Host-side construction of a codebook (CPU float32 tensor)."""
@@ -283,9 +295,8 @@ def bnbq_step_8bit(opt: str | int, tensors: Sequence[TensorState] | ctypes.Array
     else:
         arr, nt = pack_tensor_list(tensors), len(tensors)
     hp = CHParams(lr, beta1, beta2, eps, weight_decay)
-    _check(lib().bnbq_step_8bit(o, arr, nt, ctypes.byref(hp), step,
-                                code1.data_ptr() if code1 is not None else None,
-                                code2.data_ptr() if code2 is not None else None, blocksize, _stream(stream)))
+    c1, c2 = _step_code(code1, "code1", None), _step_code(code2, "code2", None)
+    _check(lib().bnbq_step_8bit(o, arr, nt, ctypes.byref(hp), step, c1, c2, blocksize, _stream(stream)))
 
 
 def bnbq_step_8bit_noalloc(opt: str | int, tensors: Sequence[TensorState] | ctypes.Array, *, lr: float,
@@ -304,10 +315,8 @@ def bnbq_step_8bit_noalloc(opt: str | int, tensors: Sequence[TensorState] | ctyp
     else:
         arr, nt = pack_tensor_list(tensors), len(tensors)
     hp = CHParams(lr, beta1, beta2, eps, weight_decay)
-    _check(lib().bnbq_step_8bit_noalloc(o, arr, nt, ctypes.byref(hp), step,
-                                        code1.data_ptr() if code1 is not None else None,
-                                        code2.data_ptr() if code2 is not None else None, blocksize,
-                                        _stream(stream)))
+    c1, c2 = _step_code(code1, "code1", None), _step_code(code2, "code2", None)
+    _check(lib().bnbq_step_8bit_noalloc(o, arr, nt, ctypes.byref(hp), step, c1, c2, blocksize, _stream(stream)))
 
 
 def bnbq_device_flags(clear: bool = False) -> int:

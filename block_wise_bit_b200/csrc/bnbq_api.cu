@@ -100,6 +100,54 @@ bnbq_status sm_count(int* out)
     return BNBQ_OK;
 }
 
+namespace {
+// cuMemGetAddressRange (driver API, v2 signature), fetched through the runtime so the library
+// needs no link against libcuda; null if unavailable.
+typedef int (*AddressRangeFn)(unsigned long long* base, size_t* size, unsigned long long ptr);
+AddressRangeFn address_range_fn()
+{
+    static AddressRangeFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<AddressRangeFn>(f);
+    }();
+    return fn;
+}
+}  // namespace
+
+bnbq_status check_device_array(const void* p, size_t bytes, const char* name)
+{
+    int dev = 0;
+    bnbq_status st = current_device(&dev);
+    if (st != BNBQ_OK) return st;
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();  // a failed query leaves a (non-sticky) error behind; clear it
+        return fail(BNBQ_EINVAL, "%s: not a CUDA device pointer (%s)", name, cudaGetErrorString(e));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(BNBQ_EINVAL, "%s: must be device memory of the current device (it is %s memory)", name,
+                    attr.type == cudaMemoryTypeHost ? "page-locked host" : "ordinary host");
+    if (attr.type == cudaMemoryTypeDevice && attr.device != dev)
+        return fail(BNBQ_EINVAL, "%s: lives on device %d but the current device is %d", name, attr.device, dev);
+    if (AddressRangeFn range = address_range_fn()) {
+        unsigned long long base = 0;
+        size_t size = 0;
+        if (range(&base, &size, reinterpret_cast<unsigned long long>(p)) == 0) {
+            const unsigned long long a = reinterpret_cast<unsigned long long>(p);
+            if (a + bytes > base + size)
+                return fail(BNBQ_EINVAL, "%s: %zu bytes from this pointer run past the end of its allocation", name, bytes);
+        } else {
+            cudaGetLastError();
+        }
+    }
+    return BNBQ_OK;
+}
+
 // ------------------------------------------------------------------------------------------
 // argument checks
 // ------------------------------------------------------------------------------------------
@@ -406,6 +454,8 @@ bnbq_status bnbq_quantize_blockwise(const float* code, int code_size, const void
     if (!aligned(A, dtype_align(a_dtype))) return fail(BNBQ_EINVAL, "A not %d-byte aligned", (int)dtype_align(a_dtype));
     if (!aligned(absmax, 4)) return fail(BNBQ_EINVAL, "absmax not 4-byte aligned");
     if (!aligned(out, code_size == 256 ? 4 : 2)) return fail(BNBQ_EINVAL, "out not %d-byte aligned", code_size == 256 ? 4 : 2);
+    st = check_device_array(code, sizeof(float) * (size_t)code_size, "code");
+    if (st != BNBQ_OK) return st;
     return launch_quantize(code, code_size, A, a_dtype, n, blocksize, absmax, out,
                            reinterpret_cast<cudaStream_t>(stream));
 }
@@ -422,6 +472,8 @@ bnbq_status bnbq_dequantize_blockwise(const float* code, int code_size, const ui
     if (!aligned(q, code_size == 256 ? 4 : 2)) return fail(BNBQ_EINVAL, "q not %d-byte aligned", code_size == 256 ? 4 : 2);
     if (!aligned(absmax, 4)) return fail(BNBQ_EINVAL, "absmax not 4-byte aligned");
     if (!aligned(out, dtype_align(out_dtype))) return fail(BNBQ_EINVAL, "out not %d-byte aligned", (int)dtype_align(out_dtype));
+    st = check_device_array(code, sizeof(float) * (size_t)code_size, "code");
+    if (st != BNBQ_OK) return st;
     return launch_dequantize(code, code_size, q, absmax, n, blocksize, out, out_dtype,
                              reinterpret_cast<cudaStream_t>(stream));
 }
@@ -486,6 +538,11 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
         if (!aligned(code1, 4) || (two && !aligned(code2, 4))) return fail(BNBQ_EINVAL, "codebook not 4-byte aligned");
     }
     if (descs.empty()) return BNBQ_OK;
+    if (any8) {  // the codebooks must be device memory of this device (checked before any launch)
+        bnbq_status cst = check_device_array(code1, 256 * sizeof(float), "code1");
+        if (cst == BNBQ_OK && two) cst = check_device_array(code2, 256 * sizeof(float), "code2");
+        if (cst != BNBQ_OK) return cst;
+    }
 
     // Scalars derived once on the host in double and rounded once to binary32.
     StepScalars sc;
@@ -509,6 +566,7 @@ bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int ntensors
     sc.lr = hp->lr;
     sc.eps = hp->eps;
     sc.wd = hp->weight_decay;
+    sc.upd_fast = update_fast_allowed(sc.eps, sc.sqrt_bc2) ? 1 : 0;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     bnbq_status st = refuse_capture(s);

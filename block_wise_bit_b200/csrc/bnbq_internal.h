@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "../../include/bnbq.h"
@@ -14,6 +15,10 @@ bnbq_status fail(bnbq_status st, const char* fmt, ...);
 bnbq_status cuda_status(cudaError_t e, const char* what);
 // BNBQ_EUNSUPPORTED if `s` is being captured into a CUDA graph (the step entry points refuse it).
 bnbq_status refuse_capture(cudaStream_t s);
+
+// BNBQ_OK if `bytes` bytes from `p` are device (or managed) memory of the current device, inside
+// one allocation; else BNBQ_EINVAL naming `name`.  Used for codebooks before any launch.
+bnbq_status check_device_array(const void* p, size_t bytes, const char* name);
 
 // Device-side flag word of the current device (a __device__ variable; its address is taken
 // once per device).
@@ -58,6 +63,12 @@ struct alignas(16) StepDesc {
     int32_t flags;        // bit 0: g is bf16; bit 1: 8-bit state
 };
 static_assert(sizeof(StepDesc) == 64, "descriptor layout");
+// The step kernel reads a descriptor as four 16-byte words (load_cur in bnbq_step.cu).
+static_assert(offsetof(StepDesc, p) == 0 && offsetof(StepDesc, g) == 8 && offsetof(StepDesc, s1) == 16 &&
+                  offsetof(StepDesc, s2) == 24 && offsetof(StepDesc, a1) == 32 && offsetof(StepDesc, a2) == 40 &&
+                  offsetof(StepDesc, n) == 48 && offsetof(StepDesc, first_block) == 56 &&
+                  offsetof(StepDesc, flags) == 60,
+              "descriptor field offsets");
 constexpr int32_t kDescGBf16 = 1;
 constexpr int32_t kDescState8 = 2;
 
@@ -69,7 +80,16 @@ struct StepScalars {
     float rcp_sqrt_bc2;  // RN(1 / sqrt_bc2)
     float decay;         // 1 - lr*wd (AdamW, Lion) or 1
     float lr, eps, wd;
+    int upd_fast;        // the FMA square root and division of the update may be used (see below)
 };
+
+// Host rule for StepScalars::upd_fast: the update's exact FMA square root and division need the
+// denominator sqrt(v)/sqrt(1-b2^t) + eps (or sqrt(v) + eps) inside [2^-50, 2^63] whenever v lies in
+// [2^-100, 2^100], which holds for 0 <= eps <= 2^60 and sqrt(1-b2^t) in [2^-12, 1].
+inline bool update_fast_allowed(float eps, float sqrt_bc2)
+{
+    return eps >= 0.0f && eps <= 0x1p60f && sqrt_bc2 >= 0x1p-12f && sqrt_bc2 <= 1.0f;
+}
 
 bnbq_status launch_step(bnbq_optim opt, const StepDesc* d_table, int ntensors, int total_blocks,
                         const StepScalars& sc, const float* code1, const float* code2, int B,

@@ -110,7 +110,9 @@ extern "C" BNBQ_API bnbq_status bnbq_quantize_absmax_nested(const float* absmax,
     if (!aligned_n(qabs, 4)) return fail(BNBQ_EINVAL, "qabs not 4-byte aligned");
     if (!aligned_n(absmax2, 4)) return fail(BNBQ_EINVAL, "absmax2 not 4-byte aligned");
     if (!aligned_n(workspace, 8)) return fail(BNBQ_EINVAL, "workspace not 8-byte aligned");
-    bnbq_status st = launch_absmax_mean(absmax, nb, static_cast<double*>(workspace), offset, s);
+    bnbq_status st = check_device_array(code2, 256 * sizeof(float), "code2");
+    if (st != BNBQ_OK) return st;
+    st = launch_absmax_mean(absmax, nb, static_cast<double*>(workspace), offset, s);
     if (st != BNBQ_OK) return st;
     return launch_quantize_centred(code2, absmax, nb, offset, absmax2, qabs, s);
 }
@@ -125,6 +127,8 @@ extern "C" BNBQ_API bnbq_status bnbq_dequantize_absmax_nested(const uint8_t* qab
         return fail(BNBQ_EINVAL, "qabs, absmax2, offset, code2 and absmax_out must be non-NULL");
     if (!aligned_n(absmax2, 4) || !aligned_n(offset, 4) || !aligned_n(code2, 4) || !aligned_n(absmax_out, 4))
         return fail(BNBQ_EINVAL, "absmax2, offset, code2 and absmax_out must be 4-byte aligned");
+    bnbq_status st = check_device_array(code2, 256 * sizeof(float), "code2");
+    if (st != BNBQ_OK) return st;
     return launch_unnest(qabs, absmax2, offset, code2, nb, absmax_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -147,6 +151,9 @@ extern "C" BNBQ_API bnbq_status bnbq_dequantize_blockwise_nested(const float* co
     if (!aligned_n(absmax2, 4) || !aligned_n(offset, 4)) return fail(BNBQ_EINVAL, "absmax2 / offset not 4-byte aligned");
     const uintptr_t oa = out_dtype == BNBQ_BF16 ? 8 : 16;
     if (!aligned_n(out, oa)) return fail(BNBQ_EINVAL, "out not %d-byte aligned", (int)oa);
+    bnbq_status st = check_device_array(code, sizeof(float) * (size_t)code_size, "code");
+    if (st == BNBQ_OK) st = check_device_array(code2, 256 * sizeof(float), "code2");
+    if (st != BNBQ_OK) return st;
     return launch_dequantize_nested(code, code_size, q, qabs, absmax2, offset, code2, n, blocksize, out, out_dtype,
                                     reinterpret_cast<cudaStream_t>(stream));
 }

@@ -12,8 +12,12 @@
 //
 // Set-up: the array's name is only a host-side stand-in for the device object, so its device
 // address is looked up with cudaGetSymbolAddress once per device (with that device current),
-// on the first call made on that device.  That first call also sets the step kernel's shared
-// memory attribute; make it before capturing any stream.
+// on the first call made on that device.  With CUDA's lazy module loading that first lookup may
+// also load the library's device code onto the device, which is when the 256 KiB table (and
+// the code) take device memory; the step kernel's shared-memory limit is likewise set up at the
+// first step call on a device for each optimizer and blocksize.  A caller that must not allocate
+// later should therefore make one call at start-up on each device it uses, and make it before
+// capturing any stream.
 //
 // Sharing: every call on a device writes its table into the same array, which keeps the last
 // call's contents.  Two calls whose work overlaps on the GPU (different streams, no ordering
@@ -128,6 +132,11 @@ extern "C" BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnb
         if (!aligned_na(code1, 4) || (two && !aligned_na(code2, 4))) return fail(BNBQ_EINVAL, "codebook not 4-byte aligned");
     }
     if (nd == 0) return BNBQ_OK;
+    if (any8) {  // the codebooks must be device memory of this device (checked before any launch)
+        bnbq_status cst = check_device_array(code1, 256 * sizeof(float), "code1");
+        if (cst == BNBQ_OK && two) cst = check_device_array(code2, 256 * sizeof(float), "code2");
+        if (cst != BNBQ_OK) return cst;
+    }
 
     // Scalars formed in double and rounded once to binary32 (same rule as bnbq_step_8bit).
     StepScalars sc;
@@ -147,6 +156,7 @@ extern "C" BNBQ_API bnbq_status bnbq_step_8bit_noalloc(bnbq_optim opt, const bnb
     sc.lr = hp->lr;
     sc.eps = hp->eps;
     sc.wd = hp->weight_decay;
+    sc.upd_fast = update_fast_allowed(sc.eps, sc.sqrt_bc2) ? 1 : 0;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     bnbq_status st = refuse_capture(s);

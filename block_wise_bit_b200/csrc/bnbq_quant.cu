@@ -96,8 +96,8 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
         if (e >= n) continue;
         float2 x0 = make_float2(v[j][0], v[j][1]), x1 = make_float2(v[j][2], v[j][3]);
         if (FAST) {
-            x0 = div2_markstein(x0, r, na);
-            x1 = div2_markstein(x1, r, na);
+            x0 = div2_rcp(x0, r, na);
+            x1 = div2_rcp(x1, r, na);
         } else {
             x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
             x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));

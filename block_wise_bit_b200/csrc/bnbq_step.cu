@@ -24,6 +24,9 @@
 // Roofline: HBM.  AdamW with 8-bit state and bf16 gradients moves 14 bytes per element
 // (p read+write 8, g 2, q1 and q2 read+write 4) plus 16 bytes per block of scales.
 #include <float.h>
+#include <limits.h>
+
+#include <mutex>
 
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
@@ -79,28 +82,24 @@ __device__ __forceinline__ Pairs make_pairs(const StepScalars& sc)
     return q;
 }
 
-// One pair of elements of the update.  Every binary32 operation is rounded on its own, in the
-// order the header documents; p - c*u is formed as p + (-c)*u, which rounds identically.
-// sqrt(v)/sqrt(1-b2^t) uses the FMA quotient: the host rejects sqrt(1-b2^t) outside [2^-60, 1]
-// (any binary32 b2 < 1 gives at least 2^-12), and sqrt(v) is 0 or at least 2^-75, so the
-// quotient is the correctly rounded one.
+// The update of one pair of elements, in two parts.  Every binary32 operation is rounded on its
+// own, in the order the header documents; p - c*u is formed as p + (-c)*u, which rounds
+// identically.
+//
+// Part 1 (states2): the new optimizer states from the old ones and g.  Lion and momentum, whose
+// parameter update needs no square root or division, also update p here.  Afterwards `m` and `v`
+// hold what part 2 reads: AdamW/Adam m' and v'; RMSprop v' (its one state) and the gradient
+// (with weight decay added) in `v`.
 template <int OPT>
-__device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, float2& p, float2 g,
+__device__ __forceinline__ void states2(const StepScalars& sc, const Pairs& k, float2& p, float2 g,
                                         float2& m, float2& v)
 {
     if constexpr (OPT == BNBQ_ADAMW || OPT == BNBQ_ADAM) {
         if constexpr (OPT == BNBQ_ADAM) {
             if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
         }
-        const float2 m1 = add2(mul2(k.b1, m), mul2(k.omb1, g));
-        const float2 v1 = add2(mul2(k.b2, v), mul2(mul2(k.omb2, g), g));
-        if constexpr (OPT == BNBQ_ADAMW) p = mul2(p, k.decay);
-        const float2 s = make_float2(__fsqrt_rn(v1.x), __fsqrt_rn(v1.y));
-        const float2 den = add2(div2_markstein(s, k.rcp_sqrt_bc2, k.nsqrt_bc2), k.eps);
-        const float2 u = make_float2(__fdiv_rn(m1.x, den.x), __fdiv_rn(m1.y, den.y));
-        p = add2(p, mul2(k.nstep, u));
-        m = m1;
-        v = v1;
+        m = add2(mul2(k.b1, m), mul2(k.omb1, g));
+        v = add2(mul2(k.b2, v), mul2(mul2(k.omb2, g), g));
     } else if constexpr (OPT == BNBQ_LION) {
         const float2 c = add2(mul2(k.b1, m), mul2(k.omb1, g));
         const float2 sg = make_float2((c.x > 0.0f) ? 1.0f : ((c.x < 0.0f) ? -1.0f : 0.0f),
@@ -115,12 +114,58 @@ __device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, f
         m = m1;
     } else {  // RMSprop: the one state (m) is the running mean of squares, b1 = alpha
         if (sc.wd != 0.0f) g = add2(g, mul2(k.wd, p));
-        const float2 v1 = add2(mul2(k.b1, m), mul2(mul2(k.omb1, g), g));
-        const float2 den = add2(make_float2(__fsqrt_rn(v1.x), __fsqrt_rn(v1.y)), k.eps);
-        const float2 u = make_float2(__fdiv_rn(g.x, den.x), __fdiv_rn(g.y, den.y));
-        p = add2(p, mul2(k.nlr, u));
-        m = v1;
+        m = add2(mul2(k.b1, m), mul2(mul2(k.omb1, g), g));
+        v = g;
     }
+}
+
+// Optimizers whose parameter update takes a square root and a division (part 2).
+template <int OPT>
+constexpr bool kHasPart2 = (OPT == BNBQ_ADAMW || OPT == BNBQ_ADAM || OPT == BNBQ_RMSPROP);
+
+// Part 2: the parameter update from part 1's (m, v).  FAST takes the FMA square root and
+// division, which are exact when the square root's operand lies in [kSqrtOpLo, kSqrtOpHi] and
+// the numerator's magnitude in [kDivNumLo, kDivNumHi] (the caller checks; with those, the host's
+// checks eps <= 2^60 and sqrt(1-b2^t) in [2^-12, 1] keep the denominator in [2^-50, 2^63] and the
+// quotient's magnitude in [2^-123, 2^110]); otherwise the IEEE intrinsics.
+// sqrt(v)/sqrt(1-b2^t) always uses the FMA quotient: the host rejects sqrt(1-b2^t) outside
+// [2^-60, 1] (any binary32 b2 < 1 gives at least 2^-12), and sqrt(v) is 0 or at least 2^-75, so
+// the quotient is the correctly rounded one.
+template <int OPT, bool FAST>
+__device__ __forceinline__ void p_update2(const Pairs& k, float2& p, float2 m, float2 v)
+{
+    if constexpr (OPT == BNBQ_ADAMW || OPT == BNBQ_ADAM) {
+        if constexpr (OPT == BNBQ_ADAMW) p = mul2(p, k.decay);
+        const float2 s = FAST ? sqrt2_ranged(v) : make_float2(__fsqrt_rn(v.x), __fsqrt_rn(v.y));
+        const float2 den = add2(div2_rcp(s, k.rcp_sqrt_bc2, k.nsqrt_bc2), k.eps);
+        const float2 u = FAST ? div2_ranged(m, den) : make_float2(__fdiv_rn(m.x, den.x), __fdiv_rn(m.y, den.y));
+        p = add2(p, mul2(k.nstep, u));
+    } else if constexpr (OPT == BNBQ_RMSPROP) {  // m = v', v = g
+        const float2 s = FAST ? sqrt2_ranged(m) : make_float2(__fsqrt_rn(m.x), __fsqrt_rn(m.y));
+        const float2 den = add2(s, k.eps);
+        const float2 u = FAST ? div2_ranged(v, den) : make_float2(__fdiv_rn(v.x, den.x), __fdiv_rn(v.y, den.y));
+        p = add2(p, mul2(k.nlr, u));
+    }
+}
+
+// Both parts with the IEEE square root and division (32-bit state path).
+template <int OPT>
+__device__ __forceinline__ void update2(const StepScalars& sc, const Pairs& k, float2& p, float2 g,
+                                        float2& m, float2& v)
+{
+    states2<OPT>(sc, k, p, g, m, v);
+    if constexpr (kHasPart2<OPT>) p_update2<OPT, false>(k, p, m, v);
+}
+
+// Range test for the FAST part 2, from the extremes of the operands over the thread's elements
+// (hi1/lo1: largest/smallest |m|, hi2/lo2: the same for v).
+template <int OPT>
+__device__ __forceinline__ bool part2_in_range(float hi1, float lo1, float hi2, float lo2)
+{
+    if constexpr (OPT == BNBQ_RMSPROP)  // m is the square root's operand, v the numerator
+        return hi1 <= kSqrtOpHi && lo1 >= kSqrtOpLo && hi2 <= kDivNumHi && lo2 >= kDivNumLo;
+    else
+        return hi1 <= kDivNumHi && lo1 >= kDivNumLo && hi2 <= kSqrtOpHi && lo2 >= kSqrtOpLo;
 }
 
 // ---- codebook tables of the step kernel ---------------------------------------------------------
@@ -209,10 +254,27 @@ __device__ __forceinline__ void store_q4(uint8_t* q, int64_t e, int64_t n, uint3
 
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return __byte_perm(w, 0u, 0x4440u + (uint32_t)i); }
 
-// Group-wide max of (x, y) over the G threads of one block-group.
+#ifndef BNBQ_DEQ_ADDR
+#define BNBQ_DEQ_ADDR 0
+#endif
+// code[byte i of w] (i a compile-time constant in the unrolled loops).
+__device__ __forceinline__ float code_at(const float* code, uint32_t w, int i)
+{
+#if BNBQ_DEQ_ADDR
+    const uint32_t off = (i == 0 ? (w << 2) : (w >> (8 * i - 2))) & 0x3fcu;  // 4 * byte i
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(code) + off);
+#else
+    return code[byte_of(w, i)];
+#endif
+}
+
+// Group-wide max of (x, y) over the G threads of one block-group, in two halves so that work
+// independent of the result can run between them: group_max_publish reduces inside each warp
+// (and, for groups of several warps, stores the warp's maxima to shared memory, double-buffered
+// by `parity`); group_max_collect waits at the group's named barrier and combines the warps.
 template <int G, int NC>
-__device__ __forceinline__ void group_max2(float& x, float& y, int gi, int tg, int lane, unsigned gmask,
-                                           float* red, int& parity)
+__device__ __forceinline__ void group_max_publish(float& x, float& y, int gi, int tg, int lane, unsigned gmask,
+                                                  float* red, int parity)
 {
     if constexpr (G <= 32) {
         x = group_max_nan<G>(x, gmask);
@@ -227,6 +289,15 @@ __device__ __forceinline__ void group_max2(float& x, float& y, int gi, int tg, i
             r[w] = x;
             if constexpr (NC == 2) r[W + w] = y;
         }
+    }
+}
+
+template <int G, int NC>
+__device__ __forceinline__ void group_max_collect(float& x, float& y, int gi, float* red, int& parity)
+{
+    if constexpr (G > 32) {
+        constexpr int W = G / 32;
+        const float* r = red + ((gi * 2 + parity) * 2) * W;
         group_barrier(1 + gi, G);
 #pragma unroll
         for (int i = 0; i < W; i++) {
@@ -252,19 +323,20 @@ struct Cur {
 
 __device__ __forceinline__ void load_cur(Cur& c, const StepDesc* __restrict__ table, int i, int ntensors)
 {
-    const StepDesc* d = table + i;
-    auto ptr = [](const void* field) {
-        return reinterpret_cast<void*>(__ldg(reinterpret_cast<const unsigned long long*>(field)));
+    const uint4* d = reinterpret_cast<const uint4*>(table + i);
+    const uint4 w0 = __ldg(d), w1 = __ldg(d + 1), w2 = __ldg(d + 2), w3 = __ldg(d + 3);
+    auto ptr = [](uint32_t lo, uint32_t hi) {
+        return reinterpret_cast<void*>(((unsigned long long)hi << 32) | lo);
     };
-    c.p = static_cast<float*>(ptr(&d->p));
-    c.g = ptr(&d->g);
-    c.q1 = static_cast<uint8_t*>(ptr(&d->s1));
-    c.q2 = static_cast<uint8_t*>(ptr(&d->s2));
-    c.a1 = static_cast<float*>(ptr(&d->a1));
-    c.a2 = static_cast<float*>(ptr(&d->a2));
-    c.n = __ldg(reinterpret_cast<const long long*>(&d->n));
-    c.first = __ldg(&d->first_block);
-    c.flags = __ldg(&d->flags);
+    c.p = static_cast<float*>(ptr(w0.x, w0.y));
+    c.g = ptr(w0.z, w0.w);
+    c.q1 = static_cast<uint8_t*>(ptr(w1.x, w1.y));
+    c.q2 = static_cast<uint8_t*>(ptr(w1.z, w1.w));
+    c.a1 = static_cast<float*>(ptr(w2.x, w2.y));
+    c.a2 = static_cast<float*>(ptr(w2.z, w2.w));
+    c.n = (int64_t)(((unsigned long long)w3.y << 32) | w3.x);
+    c.first = (int)w3.z;
+    c.flags = (int)w3.w;
 }
 
 // Requantize the kNCH chunks of one block: FAST selects the FMA quotient; M1 / M2 are the
@@ -288,12 +360,12 @@ __device__ __forceinline__ void requant(const Cur& c, int64_t base, int tg, cons
         uint32_t w1[4], w2[4];
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            const float2 xn = FAST ? div2_markstein(mv[2 * j + h], r1, na1)
+            const float2 xn = FAST ? div2_rcp(mv[2 * j + h], r1, na1)
                                    : make_float2(__fdiv_rn(mv[2 * j + h].x, s1.a), __fdiv_rn(mv[2 * j + h].y, s1.a));
             w1[2 * h] = step_code_word<M1>(t1, mid1, xn.x);
             w1[2 * h + 1] = step_code_word<M1>(t1, mid1, xn.y);
             if constexpr (TWO) {
-                const float2 yn = FAST ? div2_markstein(vv[2 * j + h], r2, na2)
+                const float2 yn = FAST ? div2_rcp(vv[2 * j + h], r2, na2)
                                        : make_float2(__fdiv_rn(vv[2 * j + h].x, s2.a), __fdiv_rn(vv[2 * j + h].y, s2.a));
                 w2[2 * h] = step_code_word<M2>(t2, mid2, yn.x);
                 w2[2 * h + 1] = step_code_word<M2>(t2, mid2, yn.y);
@@ -351,6 +423,7 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     constexpr int G = SGeom<B>::G;
     constexpr bool TWO = OptTraits<OPT>::kTwoStates;
     constexpr int NC = OptTraits<OPT>::kCodes;
+    constexpr bool P2 = kHasPart2<OPT>;
     const float* code1 = cs.code[0];
     const float* code2 = cs.code[NC - 1];
     const int64_t n = c.n;
@@ -373,28 +446,59 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     const float a2 = TWO ? __ldg(c.a2 + lb) : 0.0f;
     const float2 a1p = f2(a1), a2p = f2(a2);
 
-    // a4 + a5: dequantize, update, store p
+    // a4 + a5: dequantize, new states, parameter update; store p
     float2 mv[2 * kNCH], vv[2 * kNCH];
-    float mx1 = 0.0f, mx2 = 0.0f;
+    float mx1 = 0.0f, mx2 = 0.0f;  // block absmax partials
+    // Running extremes of part 2's operands (|m|, |v|) over the thread's chunks so far: part 2 of a
+    // chunk takes the FMA square root and division when they lie in the exact range for every
+    // thread of the warp (one warp-uniform choice per chunk).
+    float lo1 = __int_as_float(0x7f800000), lo2 = lo1, hi2 = 0.0f;
 #pragma unroll
     for (int j = 0; j < kNCH; j++) {
         const int64_t e = e0 + 4 * G * j;
         float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            float2 m = mul2(make_float2(code1[byte_of(w1[j], 2 * h)], code1[byte_of(w1[j], 2 * h + 1)]), a1p);
+            float2 m = mul2(make_float2(code_at(code1, w1[j], 2 * h), code_at(code1, w1[j], 2 * h + 1)), a1p);
             float2 v = make_float2(0.0f, 0.0f);
             if constexpr (TWO)
-                v = mul2(make_float2(code2[byte_of(w2[j], 2 * h)], code2[byte_of(w2[j], 2 * h + 1)]), a2p);
-            update2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
+                v = mul2(make_float2(code_at(code2, w2[j], 2 * h), code_at(code2, w2[j], 2 * h + 1)), a2p);
+            states2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
             if (!FULL) {  // elements past the end do not count towards the block scale
                 if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }
                 if (e + 2 * h + 1 >= n) { m.y = 0.0f; v.y = 0.0f; }
             }
             mv[2 * j + h] = m;
             vv[2 * j + h] = v;
+#if BNBQ_MINMAX3
+            mx1 = max3_abs_nan(mx1, m.x, m.y);
+            if constexpr (TWO) mx2 = max3_abs_nan(mx2, v.x, v.y);
+            if constexpr (P2 && FULL) {
+                lo1 = min3_abs(lo1, m.x, m.y);
+                lo2 = min3_abs(lo2, v.x, v.y);
+                if constexpr (!TWO) hi2 = max3_abs_nan(hi2, v.x, v.y);
+            }
+#else
             mx1 = max_nan(mx1, max_nan(fabsf(m.x), fabsf(m.y)));
             if constexpr (TWO) mx2 = max_nan(mx2, max_nan(fabsf(v.x), fabsf(v.y)));
+            if constexpr (P2 && FULL) {
+                lo1 = fminf(lo1, fminf(fabsf(m.x), fabsf(m.y)));
+                lo2 = fminf(lo2, fminf(fabsf(v.x), fabsf(v.y)));
+                if constexpr (!TWO) hi2 = max_nan(hi2, max_nan(fabsf(v.x), fabsf(v.y)));
+            }
+#endif
+        }
+        if constexpr (P2) {
+            bool fast = false;
+            if constexpr (FULL)
+                fast = __all_sync(gmask, sc.upd_fast && part2_in_range<OPT>(mx1, lo1, TWO ? mx2 : hi2, lo2));
+            if (fast) {
+                p_update2<OPT, true>(kp, ph[0], mv[2 * j], vv[2 * j]);
+                p_update2<OPT, true>(kp, ph[1], mv[2 * j + 1], vv[2 * j + 1]);
+            } else {
+                p_update2<OPT, false>(kp, ph[0], mv[2 * j], vv[2 * j]);
+                p_update2<OPT, false>(kp, ph[1], mv[2 * j + 1], vv[2 * j + 1]);
+            }
         }
         const float4 po = make_float4(ph[0].x, ph[0].y, ph[1].x, ph[1].y);
         if (FULL) {
@@ -405,16 +509,18 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
     }
 
     // a6: block absmax of the new states
-    group_max2<G, NC>(mx1, mx2, gi, tg, lane, gmask, red, parity);
+    float r1 = mx1, r2 = mx2;
+    group_max_publish<G, NC>(r1, r2, gi, tg, lane, gmask, red, parity);
+    group_max_collect<G, NC>(r1, r2, gi, red, parity);
     if (tg == 0) {
-        c.a1[lb] = mx1;
-        if constexpr (TWO) c.a2[lb] = mx2;
-        if (!(mx1 <= FLT_MAX) || !(mx2 <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
+        c.a1[lb] = r1;
+        if constexpr (TWO) c.a2[lb] = r2;
+        if (!(r1 <= FLT_MAX) || !(r2 <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
     }
 
     // a7: requantize (one block-uniform choice of quotient)
-    const BlockScale s1 = make_scale(mx1, fast1);
-    const BlockScale s2 = TWO ? make_scale(mx2, fast2) : s1;
+    const BlockScale s1 = make_scale(r1, fast1);
+    const BlockScale s2 = TWO ? make_scale(r2, fast2) : s1;
     if (s1.fast && s2.fast)
         requant<OPT, B, FULL, M1, M2, true>(c, base, tg, cs, mv, vv, s1, s2);
     else
@@ -423,7 +529,8 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
 
 // One block with 32-bit state (no quantization).
 template <int OPT, int B>
-__device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp, int tg)
+__device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScalars& sc, const Pairs& kp, int tg,
+                                        unsigned gmask)
 {
     constexpr int G = SGeom<B>::G;
     constexpr bool TWO = OptTraits<OPT>::kTwoStates;
@@ -444,8 +551,27 @@ __device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScal
         float2 ph[2] = {make_float2(pv.x, pv.y), make_float2(pv.z, pv.w)};
         float2 mh[2] = {make_float2(mq.x, mq.y), make_float2(mq.z, mq.w)};
         float2 vh[2] = {make_float2(vq.x, vq.y), make_float2(vq.z, vq.w)};
-        update2<OPT>(sc, kp, ph[0], make_float2(gv.x, gv.y), mh[0], vh[0]);
-        update2<OPT>(sc, kp, ph[1], make_float2(gv.z, gv.w), mh[1], vh[1]);
+        states2<OPT>(sc, kp, ph[0], make_float2(gv.x, gv.y), mh[0], vh[0]);
+        states2<OPT>(sc, kp, ph[1], make_float2(gv.z, gv.w), mh[1], vh[1]);
+        if constexpr (kHasPart2<OPT>) {
+            // FMA square root and division when the chunk's operands lie in their exact range for
+            // the whole warp (full blocks only, where every thread of the group takes this chunk)
+            bool fast = false;
+            if (full) {
+                const float hi1 = max_nan(max_nan(fabsf(mh[0].x), fabsf(mh[0].y)), max_nan(fabsf(mh[1].x), fabsf(mh[1].y)));
+                const float lo1 = fminf(fminf(fabsf(mh[0].x), fabsf(mh[0].y)), fminf(fabsf(mh[1].x), fabsf(mh[1].y)));
+                const float hi2 = max_nan(max_nan(fabsf(vh[0].x), fabsf(vh[0].y)), max_nan(fabsf(vh[1].x), fabsf(vh[1].y)));
+                const float lo2 = fminf(fminf(fabsf(vh[0].x), fabsf(vh[0].y)), fminf(fabsf(vh[1].x), fabsf(vh[1].y)));
+                fast = __all_sync(gmask, sc.upd_fast && part2_in_range<OPT>(hi1, lo1, hi2, lo2));
+            }
+            if (fast) {
+                p_update2<OPT, true>(kp, ph[0], mh[0], vh[0]);
+                p_update2<OPT, true>(kp, ph[1], mh[1], vh[1]);
+            } else {
+                p_update2<OPT, false>(kp, ph[0], mh[0], vh[0]);
+                p_update2<OPT, false>(kp, ph[1], mh[1], vh[1]);
+            }
+        }
         store_f4_guard(c.p, e, n, make_float4(ph[0].x, ph[0].y, ph[1].x, ph[1].y));
         store_f4_guard(m32, e, n, make_float4(mh[0].x, mh[0].y, mh[1].x, mh[1].y));
         if constexpr (TWO) store_f4_guard(v32, e, n, make_float4(vh[0].x, vh[0].y, vh[1].x, vh[1].y));
@@ -465,9 +591,15 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
     const int lane = threadIdx.x & 31;
     const unsigned gmask = (G >= 32) ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
     int parity = 0;
-    int cur = 0;
+    int cur = -1;
+    int next_first = 0;  // first block of tensor cur + 1 (INT_MAX past the last tensor)
     for (int b = blockIdx.x * Geo::kGroups + gi; b < total_blocks; b += gridDim.x * Geo::kGroups) {
-        while (cur + 1 < ntensors && __ldg(&table[cur + 1].first_block) <= b) cur++;
+        while (b >= next_first) {  // this block starts a later tensor: advance the cursor
+            cur++;
+            next_first = cur + 1 < ntensors ? __ldg(&table[cur + 1].first_block) : INT_MAX;
+        }
+        // The descriptor is re-read for every block (four 16-byte loads, L1-resident) rather than
+        // kept in registers across blocks, which the update needs.
         Cur c;
         load_cur(c, table, cur, ntensors);
         const int64_t lb = (int64_t)(b - c.first);
@@ -485,7 +617,7 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
                     block8<OPT, B, false, M1, M2, false>(c, lb, sc, kp, cs, fast1, fast2, gi, tg, lane, gmask, red, parity, flags);
             }
         } else {
-            block32<OPT, B>(c, lb, sc, kp, tg);
+            block32<OPT, B>(c, lb, sc, kp, tg, gmask);
         }
     }
 }
@@ -546,23 +678,34 @@ bnbq_status launch_step_t(const StepDesc* d_table, int ntensors, int total_block
     if (st != BNBQ_OK) return st;
     auto kern = step_kernel<OPT, B>;
     constexpr size_t smem = step_smem_bytes<OPT, B>();
-    static thread_local int cached_dev = -1, cached_per_sm = 0;
+    // The kernel's shared-memory limit and its resident CTAs per SM, set up once per device (for
+    // this optimizer and blocksize) by whichever call first launches it there.
+    constexpr int kDevs = 64;
+    static std::mutex mu;
+    static int per_sm_of[kDevs] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
-    if (cached_dev != dev) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(step smem)");
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached_per_sm, kern, Geo::kThreads, smem);
-        if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-        if (cached_per_sm < 1) return fail(BNBQ_ECUDA, "step kernel does not fit on an SM");
-        cached_dev = dev;
+    if (dev < 0 || dev >= kDevs) return fail(BNBQ_EUNSUPPORTED, "device ordinal %d", dev);
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!per_sm_of[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(step smem)");
+            int v = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, Geo::kThreads, smem);
+            if (e != cudaSuccess) return cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+            if (v < 1) return fail(BNBQ_ECUDA, "step kernel does not fit on an SM");
+            per_sm_of[dev] = v;
+        }
+        per_sm = per_sm_of[dev];
     }
     int sms = 0;
     st = sm_count(&sms);
     if (st != BNBQ_OK) return st;
     const int64_t need = ((int64_t)total_blocks + Geo::kGroups - 1) / Geo::kGroups;
-    const int64_t cap = (int64_t)sms * cached_per_sm;
+    const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(need < cap ? need : cap);
     kern<<<grid, Geo::kThreads, smem, s>>>(d_table, ntensors, total_blocks, sc, code1, code2, flags);
     return cuda_status(cudaGetLastError(), "step_kernel launch");

@@ -206,8 +206,11 @@ BNBQ_API bnbq_status bnbq_step_8bit(bnbq_optim opt, const bnbq_tensor* list, int
  * compiled into the library: at most 4096 non-empty tensors per call (256 KiB of device memory
  * on every GPU that loads the library, kept until the process exits); a longer list returns
  * BNBQ_EINVAL.  It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on
- * each device looks up the table's device address and sets the kernel's shared-memory limit.  Like
- * bnbq_step_8bit it refuses a stream that is being captured (BNBQ_EUNSUPPORTED).  All calls on a
+ * each device looks up the table's device address; with CUDA's lazy module loading that lookup may
+ * load the library's device code, which is when the table (and the code) take device memory.  A
+ * caller that must not allocate later should make one call on each device at start-up, before
+ * capturing any stream.  Like bnbq_step_8bit it refuses a stream that is being captured
+ * (BNBQ_EUNSUPPORTED).  All calls on a
  * device share the one table and each call rewrites the entries it uses: calls whose work can
  * overlap on the GPU (different streams with no ordering between them) race on it, so order them.
  */

@@ -347,3 +347,28 @@ def test_front_end_refuses_a_group_on_several_devices(monkeypatch):
     p2.grad = torch.ones(5000, device="meta")
     with pytest.raises(ValueError, match="one device"):
         O.AdamW8bit([p1, p2], lr=1e-3).step()
+
+
+def test_step_codebooks_are_checked_before_the_library_is_called(monkeypatch):
+    """The step wrappers pass a codebook to the library only if it is a contiguous float32 CUDA
+    tensor of 256 codes on the current device: a host codebook (what bnbq_codebook returns) or a
+    16-entry one is refused in Python, so the kernel never reads a host pointer or past the end
+    of a short table."""
+    import torch
+    arr = (B.CTensor * 1)(_t())
+
+    class NoLib:
+        def __getattr__(self, name):
+            pytest.fail(f"library called ({name})")
+
+    monkeypatch.setattr(B, "lib", lambda *a, **kw: NoLib())
+    hp = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, blocksize=2048)
+    for fn in (B.bnbq_step_8bit, B.bnbq_step_8bit_noalloc):
+        with pytest.raises(TypeError, match="CUDA tensor"):
+            fn("adamw", arr, ntensors=1, code1=torch.zeros(256), code2=torch.zeros(256), **hp)
+        with pytest.raises(ValueError, match="256 float32 codes"):
+            fn("adamw", arr, ntensors=1, code1=torch.zeros(16), code2=torch.zeros(256), **hp)
+        with pytest.raises(ValueError, match="256 float32 codes"):
+            fn("adamw", arr, ntensors=1, code1=torch.zeros(256, dtype=torch.float64), code2=torch.zeros(256), **hp)
+        with pytest.raises(TypeError, match="torch.Tensor"):
+            fn("lion", arr, ntensors=1, code1=[0.0] * 256, code2=None, **hp)

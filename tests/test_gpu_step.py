@@ -449,7 +449,13 @@ def _slice_state(fl, i, b0, b1):
     return bq.TensorState(ts.p[e0:e1], ts.g[e0:e1], s(ts.state1), s(ts.state2))
 
 
-def _full_size_run(shape, optim, seed, steps, picks_fn, g_outlier=(0.0, 1.0)):
+def _full_size_run(shape, optim, seed, steps, picks_fn, g_outlier=(0.0, 1.0), check_at=None):
+    """Step the whole list ``steps`` times (one launch per step) and compare the sampled block
+    ranges with the oracle.  ``check_at=None``: the oracle follows its own trajectory from the
+    same seeded start and is compared after every step.  Otherwise only at the steps in
+    ``check_at``, each from the GPU's pre-step state of those ranges copied to the host (one oracle
+    step on that state: no drift, and the states late in training are checked as they are).
+    Returns the number of elements compared and the sum of the mismatch counts."""
     if torch.cuda.get_device_properties(0).total_memory < 80e9 and shape == "llama7b":
         pytest.skip("needs a GPU with >= 80 GB")
     B = 2048
@@ -461,23 +467,32 @@ def _full_size_run(shape, optim, seed, steps, picks_fn, g_outlier=(0.0, 1.0)):
     two = optim in ("adamw", "adam")
     ranges = _sample_ranges(lay, B, picks_fn(lay))
     hosts = [HostTensor(_slice_state(fl, i, b0, b1)) for (i, b0, b1) in ranges]
+    compared = mismatches = 0
     for t in range(1, steps + 1):
         for i, spec in enumerate(lay.specs):
             W.grad_fill_(fl.entries[i].g, 1e-3, g_outlier[0], g_outlier[1], shape, seed, i, "g", t)
-        prevs = [_copy_prev(h) for h in hosts]
+        check = check_at is None or t in check_at
+        if check and check_at is not None:  # the oracle starts from the GPU's state before this step
+            torch.cuda.synchronize()
+            hosts = [HostTensor(_slice_state(fl, i, b0, b1)) for (i, b0, b1) in ranges]
+        prevs = [_copy_prev(h) for h in hosts] if check else None
         fl.step(t, **HP[optim])
         torch.cuda.synchronize()
+        if not check:
+            continue
         for (i, b0, b1), ht, prev in zip(ranges, hosts, prevs):
             ts = _slice_state(fl, i, b0, b1)
             g_np = parity.to_np(ts.g)
             parity.oracle_step_numpy(optim, ht.p, g_np, ht.s1, ht.s2, ht.a1, ht.a2, c1.numpy(),
                                      c2.numpy() if two else None, B, HP[optim], t)
-            _compare(f"{shape}/{optim}/{lay.specs[i].name}[{b0}:{b1}]", ts, ht, g_np, optim, B, t, c1.numpy(),
-                     c2.numpy() if two else None, prev)
+            mismatches += _compare(f"{shape}/{optim}/{lay.specs[i].name}[{b0}:{b1}]", ts, ht, g_np, optim, B, t,
+                                   c1.numpy(), c2.numpy() if two else None, prev)
+            compared += ht.p.size
     # property over the whole list: every 8-bit block scale is finite and non-negative
     assert bool(torch.isfinite(fl.a1).all()) and bool((fl.a1 >= 0).all())
     del fl
     torch.cuda.empty_cache()
+    return compared, mismatches
 
 
 def _gpt2_picks(lay):
@@ -505,3 +520,14 @@ def test_llama7b_one_state_full_size(optim):
 
 def test_llama7b_adamw_full_size():
     _full_size_run("llama7b", "adamw", 4, 2, _llama_picks)
+
+
+def test_llama7b_adamw_late_steps_full_size():
+    """The 7B AdamW list stepped 100 times; at steps 1, 2, 50 and 100 the sampled ranges (the
+    embedding, lm_head, one tensor of each shape class and every partial last block) are checked
+    from the GPU's own pre-step state, so states that have run many steps -- block scales shrunk
+    with the moments, codes in small-magnitude buckets -- are compared at full size."""
+    compared, mismatches = _full_size_run("llama7b", "adamw", 4, 100, _llama_picks, check_at={1, 2, 50, 100})
+    REPORT.append(f"llama7b/adamw steps 1, 2, 50, 100 from the GPU's pre-step state: {compared} elements compared, "
+                  f"{mismatches} differing values of any kind (p bits, codes, block scales)")
+    assert compared > 0

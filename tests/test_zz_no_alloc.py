@@ -97,3 +97,21 @@ def test_noalloc_rejects_lists_beyond_its_table():
     rc = B.lib().bnbq_step_8bit_noalloc(0, arr, n, ctypes.byref(hp), 1, 0x7000, 0x8000, 2048, None)
     assert rc == B.EINVAL
     assert "at most 4096" in B.bnbq_last_error()
+
+
+def test_noalloc_step_takes_no_device_memory():
+    """After one call on the device (which may load the library's device code), further calls
+    with lists of different lengths leave the device's free memory unchanged: the entry point
+    allocates nothing, not even the descriptor table that the allocating entry point caches."""
+    c1 = bq.bnbq_codebook("dynamic_signed").to(DEV)
+    c2 = bq.bnbq_codebook("dynamic_unsigned").to(DEV)
+    _, lists = _list(9, SIZES, 2048)
+    subsets = [lists, lists[:2], lists[3:], lists[1:5]]
+    B.bnbq_step_8bit_noalloc("adamw", lists, step=1, code1=c1, code2=c2, blocksize=2048, **HP)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for t, sub in enumerate(subsets, start=2):
+        B.bnbq_step_8bit_noalloc("adamw", sub, step=t, code1=c1, code2=c2, blocksize=2048, **HP)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert bq.bnbq_device_flags(clear=True) == 0
