@@ -70,19 +70,27 @@ QUANT_WORKLOADS = {
 }
 
 
-def bench_quant(args, base):
-    """Time bnbq_quantize_blockwise and bnbq_dequantize_blockwise on one sweep point (inputs far
-    above the L2 size for 2^28 elements); one JSON line with GB/s of each against the HBM peak."""
+# The sweep of standalone quantize / dequantize measurements: every combination of these.
+QUANT_SWEEP = dict(log2n=(20, 24, 28), dtype=("f32", "bf16"), code=("dynamic_signed", "nf4"),
+                   blocksize=(256, 2048, 4096))
+L2_BYTES = 126 << 20
+
+
+def quant_point(point, steps, warmup, seed_tag):
+    """Time bnbq_quantize_blockwise and bnbq_dequantize_blockwise on one point (log2 n, input dtype,
+    codebook, blocksize, nested scales); inputs ~N(0,1) with 0.1% of positions x50 (seed 1).  When
+    the point's inputs and outputs fit in L2, a 512 MB buffer is written between every timed call
+    so that each one starts from HBM.  Returns a dict of timings and fractions of the HBM peak."""
     import torch
     import block_wise_bit_b200 as bq
     from block_wise_bit_b200 import workloads as W
-    log2n, dt, code_name, B, nested = QUANT_WORKLOADS[args.workload]
+    log2n, dt, code_name, B, nested = point
     n = 1 << log2n
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     dtype = torch.float32 if dt == "f32" else torch.bfloat16
-    x = W.normal(n, 1.0, dev, "quant-sweep", 1, args.workload)
-    W.outliers_(x, 0.001, 50.0, dev, "quant-sweep", 1, args.workload)
+    x = W.normal(n, 1.0, dev, "quant-sweep", 1, seed_tag)
+    W.outliers_(x, 0.001, 50.0, dev, "quant-sweep", 1, seed_tag)
     x = x.to(dtype)
     code = bq.bnbq_codebook(code_name).to(dev)
     K = code.numel()
@@ -95,11 +103,13 @@ def bench_quant(args, base):
     alg_q = n * esz + qbytes + 4 * nb
     alg_dq = qbytes + 4 * nb + n * esz
     stream = torch.cuda.current_stream(dev)
+    code2 = None
     if nested:  # nest: read the scales twice (mean, quantize), write codes + second-level scales
         code2 = bq.bnbq_codebook("dynamic_signed").to(dev)
         nb2 = (nb + 255) // 256
         alg_q += 8 * nb + nb + 4 * nb2
         alg_dq = qbytes + nb + 4 * nb2 + n * esz
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if alg_q + alg_dq < L2_BYTES else None
 
     def quantize():
         bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
@@ -111,29 +121,55 @@ def bench_quant(args, base):
         else:
             bq.bnbq_dequantize_blockwise(code, q, absmax, n, B, out=y)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         dequantize(quantize())
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for k in range(args.steps):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        if flush is not None:
+            flush.zero_()
         evs[k][0].record(stream)
         nest = quantize()
         evs[k][1].record(stream)
-        dequantize(nest)
+        if flush is not None:
+            flush.zero_()
         evs[k][2].record(stream)
+        dequantize(nest)
+        evs[k][3].record(stream)
     torch.cuda.synchronize()
-    tq = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    td = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    tq = sorted(e[0].elapsed_time(e[1]) for e in evs)
+    td = sorted(e[2].elapsed_time(e[3]) for e in evs)
+    mq, md = statistics.median(tq), statistics.median(td)
+    peak, _ = measured_peaks()
+    return dict(n=n, dtype=dt, codebook=code_name, blocksize=B, nested_scales=nested,
+                l2="written between calls (inputs fit in L2)" if flush is not None else "inputs far larger than L2",
+                quantize={"ms": round(mq, 4), "GB/s": round(alg_q / mq / 1e6, 1),
+                          "frac": round(alg_q / mq / 1e6 / peak, 4), "bytes": int(alg_q)},
+                dequantize={"ms": round(md, 4), "GB/s": round(alg_dq / md / 1e6, 1),
+                            "frac": round(alg_dq / md / 1e6 / peak, 4), "bytes": int(alg_dq)},
+                elements_per_s=n / ((mq + md) / 1e3), launches=(5 if nested else 2) * steps)
+
+
+def bench_quant(args, base):
+    """One sweep point (--workload quant_*) or the whole sweep (--workload quant_sweep): one JSON
+    line per point with GB/s of quantize and dequantize against the HBM peak."""
+    import itertools
+    if args.workload == "quant_sweep":
+        points = [(l, d, c, b, False) for l, d, c, b in itertools.product(*QUANT_SWEEP.values())]
+    else:
+        points = [QUANT_WORKLOADS[args.workload]]
     peak, kind = measured_peaks()
-    out = dict(base, metric="block-wise quantize + dequantize elements/s", unit="elements/s",
-               value=n / ((tq + td) / 1e3), n_gpus=1, steps=args.steps, warmup=args.warmup,
-               ms_per_step=round(tq + td, 4), dtype=dt,
-               config={"workload": args.workload, "n": n, "blocksize": B, "codebook": code_name,
-                       "nested_scales": nested},
-               quantize={"ms": round(tq, 4), "GB/s": round(alg_q / tq / 1e6, 1), "frac": round(alg_q / tq / 1e6 / peak, 4)},
-               dequantize={"ms": round(td, 4), "GB/s": round(alg_dq / td / 1e6, 1), "frac": round(alg_dq / td / 1e6 / peak, 4)},
-               peak_gbs=peak, gpu_launches=(5 if nested else 2) * args.steps)
-    print(json.dumps(out))
+    for pt in points:
+        r = quant_point(pt, args.steps, args.warmup, args.workload if len(points) == 1 else "sweep")
+        out = dict(base, metric="block-wise quantize + dequantize elements/s", unit="elements/s",
+                   value=r.pop("elements_per_s"), n_gpus=1, steps=args.steps, warmup=args.warmup,
+                   ms_per_step=round(r["quantize"]["ms"] + r["dequantize"]["ms"], 4), dtype=pt[1],
+                   config={"workload": args.workload, **{k: r.pop(k) for k in ("n", "dtype", "codebook", "blocksize",
+                                                                                "nested_scales", "l2")}},
+                   quantize=r["quantize"], dequantize=r["dequantize"], peak_gbs=peak, peak_source=kind,
+                   gpu_launches=r["launches"], quantize_src_sha=quant_source_sha())
+        print(json.dumps(out), flush=True)
+
 
 def bench_zero1(args, base, shape, optim, seed, hp, outlier):
     """ZeRO-1 data-parallel step over the whole list on ``world`` ranks: every rank holds the full
@@ -275,6 +311,20 @@ def _code_only(text: str) -> str:
     return re.sub(r" *\n[\s]*", "\n", re.sub(" +", " ", "".join(out))).strip()
 
 
+QUANT_SOURCES = [os.path.join(ROOT, "block_wise_bit_b200", "csrc", f) for f in
+                 ("bnbq_quant.cu", "bnbq_nested.cu", "bnbq_device.cuh", "bnbq_internal.h")]
+
+
+def quant_source_sha() -> str:
+    """Hash of the quantize / dequantize kernels' code (comments and spacing ignored)."""
+    h = hashlib.sha256()
+    for f in QUANT_SOURCES:
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
+        h.update(b"\0")
+    return h.hexdigest()[:16]
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -398,6 +448,10 @@ def oracle_rate(shape: str, optim: str, hp: dict, elements8: int, threads: int, 
     oracle.lib()
     t0 = time.perf_counter()
     for t in range(1, steps + 1):
+        if threads == 1:  # one thread: the jobs one after another
+            for j in jobs:
+                run(j, t)
+            continue
         ths = [threading.Thread(target=run, args=(j, t)) for j in jobs]
         for th in ths:
             th.start()
@@ -440,7 +494,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS), default="llama7b_adamw")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS) + ["quant_sweep"],
+                    default="llama7b_adamw")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -457,7 +512,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.workload in QUANT_WORKLOADS:
+    if args.workload.startswith("quant"):
         shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS["llama7b_adamw"]
     else:
         shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS[args.workload]
@@ -614,7 +669,10 @@ def main():
         e_ms = max_over_ranks(e_ms, dev, world)
         e2e = {"value": whole_job_rate(lay.n_params, args.e2e_steps, world, e_ms), "unit": "params/s",
                "h2d_bytes_per_step": sum(b - a for (_, _, a, b) in slices) * g_host.element_size(),
-               "d2h_bytes_per_step": 4, "steps": args.e2e_steps, "slices": len(slices)}
+               "d2h_bytes_per_step": 4, "steps": args.e2e_steps, "slices": len(slices),
+               "scope": "each step uploads that step's bf16 gradients from pinned host memory and reads the "
+                        "device status word back; parameters and optimizer state stay resident on the device, "
+                        "as in a training loop"}
         del g_host, packed
 
     cpu = None
@@ -624,8 +682,10 @@ def main():
         if dt < args.cpu_seconds:
             k = max(2, math.ceil(args.cpu_seconds / max(dt, 1e-3)))
             r, dt, sample = oracle_rate(shape, optim, hp, args.cpu_sample, threads, k)
+        r1, dt1, sample1 = oracle_rate(shape, optim, hp, 1 << 22, 1, 1)
         cpu = {"value": r, "unit": "params/s", "cores": threads, "kind": "oracle", "sample": sample,
-               "seconds": round(dt, 2)}
+               "seconds": round(dt, 2),
+               "single_thread": {"value": r1, "unit": "params/s", "sample": sample1, "seconds": round(dt1, 2)}}
 
     if rank == 0:
         out = dict(base, value=value, n_gpus=world, steps=args.steps, warmup=args.warmup,

@@ -9,25 +9,85 @@
 // 8/64 + 32/(64*256) bits per weight for the scales instead of 32/64.
 //
 // The mean is a plain double sum in a fixed order -- chunks of kNestChunk consecutive scales,
-// each summed in index order (one CTA per chunk), then the chunk sums in index order --
-// divided by nb in double and rounded once to binary32, so every run (and the CPU restatement)
-// gets the same offset.  This is a one-off pass over nb = n/64 scales, far off the step's path.
+// each summed in index order, then the chunk sums in index order -- divided by nb in double and
+// rounded once to binary32, so every run (and the CPU restatement) gets the same offset.  A
+// chunk whose index-order sum is exact (see absmax_chunk_sums) is added up in parallel.
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 
 namespace bnbq {
 namespace {
 
-// One CTA per chunk: the chunk is staged in shared memory with coalesced loads, then one
-// thread adds it up in index order (the order is part of the definition of the offset).
-__global__ void __launch_bounds__(256)
+// min / max of an int over the CTA (every thread calls; every thread gets the result)
+__device__ __forceinline__ int min_over_block(int v)
+{
+    __shared__ int r[32];
+    for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, off));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) r[threadIdx.x >> 5] = v;
+    __syncthreads();
+    v = r[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); w++) v = min(v, r[w]);
+    return v;
+}
+
+__device__ __forceinline__ int max_over_block(int v)
+{
+    return -min_over_block(-v);
+}
+
+// One CTA per chunk: the chunk is staged in shared memory with coalesced loads and summed in
+// double.  The definition is the index-order sum, s = ((a0 + a1) + a2) + ...; when every partial
+// sum of that order is exact the result does not depend on the order, and the CTA adds in
+// parallel.  That holds when the ulps of the chunk's non-zero values span at most 2^17: every
+// value is then an integer multiple of the smallest ulp U and below 2^24 times the largest, so
+// the sum of at most 4096 = 2^12 of them stays below 2^(24+12+17) U = 2^53 U, an integer number
+// of U's that a double holds exactly.  Otherwise (a wider spread, or a NaN or infinity) one thread
+// adds in index order.
+constexpr int kSumThreads = 256;
+constexpr int kPerThread = kNestChunk / kSumThreads;  // 16 consecutive values per thread
+
+__device__ __forceinline__ int ulp_exponent(float x)  // biased exponent of x's ulp; 1 for subnormals
+{
+    const int e = (int)((__float_as_uint(x) >> 23) & 0xffu);
+    return e == 0 ? 1 : e;
+}
+
+__global__ void __launch_bounds__(kSumThreads)
 absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ work)
 {
     __shared__ float chunk[kNestChunk];
+    __shared__ double part[kSumThreads / 32];
     const int64_t start = (int64_t)blockIdx.x * kNestChunk;
     const int len = (int)((nb - start < kNestChunk) ? nb - start : kNestChunk);
     for (int i = threadIdx.x; i < len; i += blockDim.x) chunk[i] = __ldg(a + start + i);
     __syncthreads();
+    // ulp exponent range of the non-zero values (a NaN or infinity forces the ordered sum)
+    int emin = 255, emax = 0;
+    const int i0 = threadIdx.x * kPerThread;
+    for (int i = i0; i < i0 + kPerThread && i < len; i++) {
+        const float x = chunk[i];
+        if (x == 0.0f) continue;
+        const int e = ulp_exponent(x);
+        emin = min(emin, e);
+        emax = max(emax, (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u ? 1000 : e);
+    }
+    emin = __syncthreads_and(emin == 255) ? 0 : min_over_block(emin);
+    emax = max_over_block(emax);
+    const bool exact = emax - emin <= 17;
+    if (exact) {  // every order gives the same (exact) sum
+        double s = 0.0;
+        for (int i = i0; i < i0 + kPerThread && i < len; i++) s = __dadd_rn(s, (double)chunk[i]);
+        for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+        if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+            for (int w = 0; w < kSumThreads / 32; w++) t = __dadd_rn(t, part[w]);
+            work[blockIdx.x] = t;
+        }
+        return;
+    }
     if (threadIdx.x != 0) return;
     double s = 0.0;
     for (int i = 0; i < len; i++) s = __dadd_rn(s, (double)chunk[i]);

@@ -13,6 +13,8 @@
 // persistent: SMs x resident CTAs, each CTA striding over blocks.
 #include <float.h>
 
+#include <mutex>
+
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 
@@ -30,10 +32,10 @@ struct QGeom {
     static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
     static constexpr size_t kSmem = sizeof(CodeSmem) + sizeof(float) * kGroups * 2 * kGroupWarps;
 };
-template <bool BF16>
+template <bool BF16, bool FULL>
 __device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, float (&v)[4])
 {
-    if (e + 4 <= n) {
+    if (FULL || e + 4 <= n) {
         if (BF16) {
             uint2 w = ld_stream_u2(static_cast<const uint16_t*>(A) + e);
             v[0] = bf16lo_to_f32(w.x);
@@ -83,8 +85,9 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
     return true;
 }
 
-// Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division).
-template <int B, int K, int MODE, bool FAST>
+// Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division; FULL:
+// the block lies entirely inside the tensor, so no element needs a bounds check).
+template <int B, int K, int MODE, bool FAST, bool FULL>
 __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockScale& sc, const float (&v)[4][4],
                                                int64_t base, int tg, int64_t n, uint8_t* __restrict__ out)
 {
@@ -93,7 +96,7 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         const int64_t e = base + 4 * (j * G + tg);
-        if (e >= n) continue;
+        if (!FULL && e >= n) continue;
         float2 x0 = make_float2(v[j][0], v[j][1]), x1 = make_float2(v[j][2], v[j][3]);
         if (FAST) {
             x0 = div2_rcp(x0, r, na);
@@ -104,9 +107,9 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
         }
         const uint32_t w0 = nearest_code_word<MODE>(cs, x0.x), w1 = nearest_code_word<MODE>(cs, x0.y);
         const uint32_t w2 = nearest_code_word<MODE>(cs, x1.x), w3 = nearest_code_word<MODE>(cs, x1.y);
+        const uint32_t word = pack_top_bytes(w0, w1, w2, w3);  // byte i = code of element e + i
         if constexpr (K == 256) {
-            const uint32_t word = pack_top_bytes(w0, w1, w2, w3);
-            if (e + 4 <= n) {
+            if (FULL || e + 4 <= n) {
                 st_stream_u32(out + e, word);
             } else {
                 out[e] = (uint8_t)word;
@@ -114,18 +117,68 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
                 if (e + 2 < n) out[e + 2] = (uint8_t)(word >> 16);
             }
         } else {  // two 4-bit codes per byte, even element in the high nibble
-            const uint32_t q0 = w0 >> 24, q1 = w1 >> 24, q2 = w2 >> 24, q3 = w3 >> 24;
-            const uint8_t b0 = (uint8_t)((q0 << 4) | (e + 1 < n ? q1 : 0u));
-            const uint8_t b1 = (uint8_t)((q2 << 4) | (e + 3 < n ? q3 : 0u));
+            // (word << 4) | (word >> 8): byte 0 = q0 << 4 | q1 and byte 2 = q2 << 4 | q3 (codes < 16)
+            const uint32_t u = (word << 4) | (word >> 8);
             uint8_t* o = out + (e >> 1);
-            if (e + 4 <= n) {
-                *reinterpret_cast<uint16_t*>(o) = (uint16_t)(b0 | (b1 << 8));
-            } else {
-                o[0] = b0;
-                if (e + 2 < n) o[1] = b1;
+            if (FULL || e + 4 <= n) {
+                *reinterpret_cast<uint16_t*>(o) = (uint16_t)__byte_perm(u, 0u, 0x4420u);
+            } else {  // the low nibble past the end stays 0
+                const uint32_t keep = e + 1 < n ? 0xffu : 0xf0u;
+                o[0] = (uint8_t)(u & keep);
+                if (e + 2 < n) o[1] = (uint8_t)((u >> 16) & (e + 3 < n ? 0xffu : 0xf0u));
             }
         }
     }
+}
+
+// One block: loads, block absmax over the group, normalise, search, store.
+template <int B, bool BF16, int K, int MODE, bool CENTER, bool FULL>
+__device__ __forceinline__ void quantize_block(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
+                                               float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
+                                               unsigned* flags, float off, int64_t b, int gi, int tg, int lane,
+                                               unsigned gmask, int& parity)
+{
+    constexpr int G = QGeom<B>::G;
+    const int64_t base = b * B;
+    float v[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) load_chunk<BF16, FULL>(A, base + 4 * (j * G + tg), n, v[j]);
+    if constexpr (CENTER) {
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (FULL || base + 4 * (j * G + tg) + i < n) v[j][i] = __fsub_rn(v[j][i], off);
+    }
+
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        m = max3_abs_nan(m, v[j][0], v[j][1]);
+        m = max3_abs_nan(m, v[j][2], v[j][3]);
+    }
+
+    if constexpr (G <= 32) {
+        m = group_max_nan<G>(m, gmask);
+    } else {
+        constexpr int W = G / 32;
+        m = group_max_nan<32>(m, 0xffffffffu);
+        float* r = red + (gi * 2 + parity) * W;
+        if (lane == 0) r[tg >> 5] = m;
+        group_barrier(1 + gi, G);
+#pragma unroll
+        for (int w = 0; w < W; w++) m = max_nan(m, r[w]);
+        parity ^= 1;
+    }
+    if (tg == 0) {
+        absmax[b] = m;
+        if (!(m <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
+    }
+    const BlockScale sc = make_scale(m, fast);
+    if (sc.fast)
+        quantize_store<B, K, MODE, true, FULL>(cs, sc, v, base, tg, n, out);
+    else
+        quantize_store<B, K, MODE, false, FULL>(cs, sc, v, base, tg, n, out);
 }
 
 // CENTER: quantize A[i] - *center (one binary32 subtraction; fp32 input), the centred block
@@ -146,45 +199,12 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
     int parity = 0;
 
     for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb; b += (int64_t)gridDim.x * Geo::kGroups) {
-        const int64_t base = b * B;
-        float v[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) load_chunk<BF16>(A, base + 4 * (j * G + tg), n, v[j]);
-        if constexpr (CENTER) {
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-#pragma unroll
-                for (int i = 0; i < 4; i++)
-                    if (base + 4 * (j * G + tg) + i < n) v[j][i] = __fsub_rn(v[j][i], off);
-        }
-
-        float m = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 4; j++)
-#pragma unroll
-            for (int i = 0; i < 4; i++) m = max_nan(m, fabsf(v[j][i]));
-
-        if constexpr (G <= 32) {
-            m = group_max_nan<G>(m, gmask);
-        } else {
-            constexpr int W = G / 32;
-            m = group_max_nan<32>(m, 0xffffffffu);
-            float* r = red + (gi * 2 + parity) * W;
-            if (lane == 0) r[tg >> 5] = m;
-            group_barrier(1 + gi, G);
-#pragma unroll
-            for (int w = 0; w < W; w++) m = max_nan(m, r[w]);
-            parity ^= 1;
-        }
-        if (tg == 0) {
-            absmax[b] = m;
-            if (!(m <= FLT_MAX)) atomicOr(flags, kFlagNonFinite);
-        }
-        const BlockScale sc = make_scale(m, fast);
-        if (sc.fast)
-            quantize_store<B, K, MODE, true>(cs, sc, v, base, tg, n, out);
+        if ((b + 1) * B <= n)  // group-uniform: every thread of the group holds the same block
+            quantize_block<B, BF16, K, MODE, CENTER, true>(cs, fast, A, n, absmax, out, red, flags, off, b, gi, tg,
+                                                           lane, gmask, parity);
         else
-            quantize_store<B, K, MODE, false>(cs, sc, v, base, tg, n, out);
+            quantize_block<B, BF16, K, MODE, CENTER, false>(cs, fast, A, n, absmax, out, red, flags, off, b, gi, tg,
+                                                            lane, gmask, parity);
     }
 }
 
@@ -377,14 +397,21 @@ bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax,
     bnbq_status st = device_flag_ptr(&flags);
     if (st != BNBQ_OK) return st;
     auto kern = quantize_kernel<B, BF16, K, CENTER>;
-    static thread_local int configured_dev = -1;
+    // The kernel's shared-memory limit, set once per device (for this instantiation).
+    constexpr int kDevs = 64;
+    static std::mutex mu;
+    static bool configured[kDevs] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
-    if (configured_dev != dev) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::kSmem);
-        if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(quantize smem)");
-        configured_dev = dev;
+    if (dev < 0 || dev >= kDevs) return fail(BNBQ_EUNSUPPORTED, "device ordinal %d", dev);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!configured[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::kSmem);
+            if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(quantize smem)");
+            configured[dev] = true;
+        }
     }
     int grid = 0;
     st = persistent_grid(kern, kQThreads, Geo::kSmem, (n + B - 1) / B, Geo::kGroups, &grid);

@@ -38,7 +38,7 @@
 #define BNBQ_STEP_THREADS 1024       // CTA size for blocksize 256 and 4096
 #endif
 #ifndef BNBQ_STEP_THREADS_2048
-#define BNBQ_STEP_THREADS_2048 BNBQ_STEP_THREADS  // CTA size for blocksize 2048
+#define BNBQ_STEP_THREADS_2048 768   // CTA size for blocksize 2048 (80 registers: no spills)
 #endif
 #ifndef BNBQ_STEP_MIN_CTAS
 #define BNBQ_STEP_MIN_CTAS 1
@@ -254,20 +254,6 @@ __device__ __forceinline__ void store_q4(uint8_t* q, int64_t e, int64_t n, uint3
 
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return __byte_perm(w, 0u, 0x4440u + (uint32_t)i); }
 
-#ifndef BNBQ_DEQ_ADDR
-#define BNBQ_DEQ_ADDR 0
-#endif
-// code[byte i of w] (i a compile-time constant in the unrolled loops).
-__device__ __forceinline__ float code_at(const float* code, uint32_t w, int i)
-{
-#if BNBQ_DEQ_ADDR
-    const uint32_t off = (i == 0 ? (w << 2) : (w >> (8 * i - 2))) & 0x3fcu;  // 4 * byte i
-    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(code) + off);
-#else
-    return code[byte_of(w, i)];
-#endif
-}
-
 // Group-wide max of (x, y) over the G threads of one block-group, in two halves so that work
 // independent of the result can run between them: group_max_publish reduces inside each warp
 // (and, for groups of several warps, stores the warp's maxima to shared memory, double-buffered
@@ -459,10 +445,10 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
         float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            float2 m = mul2(make_float2(code_at(code1, w1[j], 2 * h), code_at(code1, w1[j], 2 * h + 1)), a1p);
+            float2 m = mul2(make_float2(code1[byte_of(w1[j], 2 * h)], code1[byte_of(w1[j], 2 * h + 1)]), a1p);
             float2 v = make_float2(0.0f, 0.0f);
             if constexpr (TWO)
-                v = mul2(make_float2(code_at(code2, w2[j], 2 * h), code_at(code2, w2[j], 2 * h + 1)), a2p);
+                v = mul2(make_float2(code2[byte_of(w2[j], 2 * h)], code2[byte_of(w2[j], 2 * h + 1)]), a2p);
             states2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
             if (!FULL) {  // elements past the end do not count towards the block scale
                 if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }
@@ -470,7 +456,6 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
             }
             mv[2 * j + h] = m;
             vv[2 * j + h] = v;
-#if BNBQ_MINMAX3
             mx1 = max3_abs_nan(mx1, m.x, m.y);
             if constexpr (TWO) mx2 = max3_abs_nan(mx2, v.x, v.y);
             if constexpr (P2 && FULL) {
@@ -478,15 +463,6 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
                 lo2 = min3_abs(lo2, v.x, v.y);
                 if constexpr (!TWO) hi2 = max3_abs_nan(hi2, v.x, v.y);
             }
-#else
-            mx1 = max_nan(mx1, max_nan(fabsf(m.x), fabsf(m.y)));
-            if constexpr (TWO) mx2 = max_nan(mx2, max_nan(fabsf(v.x), fabsf(v.y)));
-            if constexpr (P2 && FULL) {
-                lo1 = fminf(lo1, fminf(fabsf(m.x), fabsf(m.y)));
-                lo2 = fminf(lo2, fminf(fabsf(v.x), fabsf(v.y)));
-                if constexpr (!TWO) hi2 = max_nan(hi2, max_nan(fabsf(v.x), fabsf(v.y)));
-            }
-#endif
         }
         if constexpr (P2) {
             bool fast = false;

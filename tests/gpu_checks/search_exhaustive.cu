@@ -33,8 +33,9 @@ __global__ void setup(const float* code, int K, float* mid, uint32_t* table, int
     }
 }
 
-template <int MODE>
-__global__ void sweep(const uint32_t* table, const float* mid, const float* ref_mid, int K,
+// One pass over every value: the reference count is formed once per value and compared with each
+// search mode that applies (check[m] != 0), mismatches counted per mode.
+__global__ void sweep(const uint32_t* table, const float* mid, const float* ref_mid, int K, int3 check,
                       unsigned long long* bad, unsigned* first)
 {
     __shared__ float rm[256];
@@ -42,35 +43,25 @@ __global__ void sweep(const uint32_t* table, const float* mid, const float* ref_
     __syncthreads();
     const uint32_t* center = table + bnbq::kHalf;
     const uint64_t total = 2ull * kHalfValues;
-    unsigned long long n = 0;
+    unsigned long long n[3] = {0, 0, 0};
     for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
         const uint32_t bits = i < kHalfValues ? (uint32_t)i : 0x80000000u + (uint32_t)(i - kHalfValues);
         const float x = __uint_as_float(bits);
-        const uint32_t q = bnbq::nearest_code_word<MODE>(center, mid, x) >> 24;
         uint32_t r = 0;
         for (int j = 0; j < K - 1; j++) r += (x > rm[j]) ? 1u : 0u;
-        if (q != r) {
-            n++;
-            atomicCAS(first, 0xffffffffu, bits);
-        }
+        uint32_t q[3] = {r, r, r};
+        if (check.x) q[0] = bnbq::nearest_code_word<bnbq::kSearchSigned>(center, mid, x) >> 24;
+        if (check.y) q[1] = bnbq::nearest_code_word<bnbq::kSearchNonNeg>(center, mid, x) >> 24;
+        if (check.z) q[2] = bnbq::nearest_code_word<bnbq::kSearchGeneral>(center, mid, x) >> 24;
+#pragma unroll
+        for (int m = 0; m < 3; m++)
+            if (q[m] != r) {
+                n[m]++;
+                atomicCAS(&first[m], 0xffffffffu, bits);
+            }
     }
-    if (n) atomicAdd(bad, n);
-}
-
-template <int MODE>
-bool run_mode(const char* name, const uint32_t* table, const float* mid, const float* ref_mid, int K,
-              unsigned long long* d_bad, unsigned* d_first)
-{
-    cudaMemset(d_bad, 0, sizeof(*d_bad));
-    cudaMemset(d_first, 0xff, sizeof(*d_first));
-    sweep<MODE><<<148 * 8, 256>>>(table, mid, ref_mid, K, d_bad, d_first);
-    const cudaError_t e = cudaDeviceSynchronize();
-    unsigned long long bad = ~0ull;
-    unsigned first = 0;
-    cudaMemcpy(&bad, d_bad, sizeof(bad), cudaMemcpyDeviceToHost);
-    cudaMemcpy(&first, d_first, sizeof(first), cudaMemcpyDeviceToHost);
-    printf("mode %s status %s mismatches %llu first %08x\n", name, cudaGetErrorString(e), bad, first);
-    return e == cudaSuccess && bad == 0;
+    for (int m = 0; m < 3; m++)
+        if (n[m]) atomicAdd(&bad[m], n[m]);
 }
 
 }  // namespace
@@ -102,8 +93,8 @@ int main(int argc, char** argv)
     if (cudaMalloc(&d_code, 256 * sizeof(float)) != cudaSuccess || cudaMalloc(&d_mid, 256 * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&d_ref, 256 * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&d_table, bnbq::kTableSize * sizeof(uint32_t)) != cudaSuccess ||
-        cudaMalloc(&d_flags, 2 * sizeof(int)) != cudaSuccess || cudaMalloc(&d_bad, sizeof(*d_bad)) != cudaSuccess ||
-        cudaMalloc(&d_first, sizeof(*d_first)) != cudaSuccess)
+        cudaMalloc(&d_flags, 2 * sizeof(int)) != cudaSuccess || cudaMalloc(&d_bad, 3 * sizeof(*d_bad)) != cudaSuccess ||
+        cudaMalloc(&d_first, 3 * sizeof(*d_first)) != cudaSuccess)
         return 3;
     cudaMemcpy(d_code, code.data(), K * sizeof(float), cudaMemcpyHostToDevice);
     cudaMemcpy(d_ref, ref_mid.data(), (K - 1) * sizeof(float), cudaMemcpyHostToDevice);
@@ -118,9 +109,27 @@ int main(int argc, char** argv)
     printf("setup status %s general %d bad %d nonneg %d midpoints %s\n", cudaGetErrorString(e), flags[0], flags[1],
            nonneg ? 1 : 0, mids_equal ? "equal" : "DIFFER");
     bool ok = e == cudaSuccess && flags[1] == 0 && mids_equal;
-    if (ok && flags[0] == 0) ok = run_mode<bnbq::kSearchSigned>("signed", d_table, d_mid, d_ref, K, d_bad, d_first) && ok;
-    if (ok && nonneg) ok = run_mode<bnbq::kSearchNonNeg>("nonneg", d_table, d_mid, d_ref, K, d_bad, d_first) && ok;
-    if (ok) ok = run_mode<bnbq::kSearchGeneral>("general", d_table, d_mid, d_ref, K, d_bad, d_first) && ok;
+    if (ok) {
+        // the one-load rule where no bucket holds two midpoints, the non-negative rule for a
+        // codebook without negative codes, the midpoint walk always
+        const int3 check = make_int3(flags[0] == 0 ? 1 : 0, nonneg ? 1 : 0, 1);
+        cudaMemset(d_bad, 0, 3 * sizeof(*d_bad));
+        cudaMemset(d_first, 0xff, 3 * sizeof(*d_first));
+        sweep<<<148 * 8, 256>>>(d_table, d_mid, d_ref, K, check, d_bad, d_first);
+        e = cudaDeviceSynchronize();
+        unsigned long long bad[3] = {~0ull, ~0ull, ~0ull};
+        unsigned first[3] = {0, 0, 0};
+        cudaMemcpy(bad, d_bad, sizeof(bad), cudaMemcpyDeviceToHost);
+        cudaMemcpy(first, d_first, sizeof(first), cudaMemcpyDeviceToHost);
+        const char* names[3] = {"signed", "nonneg", "general"};
+        const int on[3] = {check.x, check.y, check.z};
+        for (int m = 0; m < 3; m++)
+            if (on[m]) {
+                printf("mode %s status %s mismatches %llu first %08x\n", names[m], cudaGetErrorString(e), bad[m],
+                       first[m]);
+                ok = ok && e == cudaSuccess && bad[m] == 0;
+            }
+    }
     printf("result %s\n", ok ? "ok" : "FAIL");
     return ok ? 0 : 1;
 }

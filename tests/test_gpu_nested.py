@@ -49,6 +49,23 @@ def test_nest_absmax_bit_exact(nb):
     np.testing.assert_array_equal(parity.to_np(r).view(np.uint32), r_or.view(np.uint32))
 
 
+@pytest.mark.parametrize("nb", [4096, 70001])
+def test_nest_absmax_mean_any_spread(nb):
+    """The mean's chunk sums: chunks whose scales span at most 2^17 in ulp size are added in
+    parallel (the index-order sum is then exact), wider ones in index order.  Chunks of both kinds,
+    zeros and subnormal scales: the offset must still equal the oracle's index-order sum."""
+    code2 = bq.bnbq_codebook("dynamic_signed")
+    a = W.log_uniform(nb, 1e-4, 1.0, DEV, "nested-spread", nb)
+    a[4096:8192] = W.log_uniform(min(4096, max(0, nb - 4096)), 1e-44, 1.0, DEV, "nested-wide", nb)  # subnormals too
+    a[::97] = 0.0
+    a[5] = 2.0 ** -130  # a subnormal in the first (narrow) chunk
+    qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2.to(DEV), a)
+    q_or, a2_or, off_or = oracle.nest_absmax(parity.to_np(a), code2.numpy())
+    assert parity.to_np(off).view(np.uint32)[0] == np.float32(off_or).view(np.uint32)
+    np.testing.assert_array_equal(parity.to_np(qabs), q_or)
+    np.testing.assert_array_equal(parity.to_np(a2).view(np.uint32), a2_or.view(np.uint32))
+
+
 def test_nest_empty_and_equal_scales():
     code2 = bq.bnbq_codebook("dynamic_signed").to(DEV)
     qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2, torch.empty(0, device=DEV))
