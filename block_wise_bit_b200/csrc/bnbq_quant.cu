@@ -2,9 +2,10 @@
 //
 // Block-wise quantization ("8-bit Optimizers via Block-wise Quantization", abstract, quoted on
 // the blog.csdn.net bitsandbytes guide, section 2): blocks of B consecutive elements are
-// scaled by their own absolute maximum and quantized independently; here one group of B/16
-// threads owns one block (16 elements per thread, as four 4-element chunks whose addresses are
-// consecutive across the group, so every load and store is a fully coalesced vector access).
+// scaled by their own absolute maximum and quantized independently; here one group of threads
+// owns one block (16 elements per thread for fp32 input, 32 for bf16, as 4-element chunks whose
+// addresses are consecutive across the group, so every load and store is a coalesced vector
+// access).
 // NF4 packing (two 4-bit codes per byte) follows the 4-bit type of the page "Bitsandbytes",
 // section "Normal Float 4 (NF4)".
 //
@@ -21,29 +22,45 @@
 namespace bnbq {
 namespace {
 
-constexpr int kEPT = 16;  // elements per thread per block
-
 constexpr int kQThreads = 512;
 
-template <int B>
+// Geometry of the quantize kernel.  A thread holds EPT elements of its group's block -- 16 for
+// fp32 input, 32 for bf16, so that every thread has 64 bytes of input in flight -- as NCH chunks
+// of CW consecutive elements (one vector load each: 4 fp32 or bf16, or 8 bf16 when WIDE); chunk
+// j of thread tg starts at element CW * (j * G + tg) of the block, so a group's loads and stores
+// are contiguous.
+template <int B, bool BF16, bool WIDE>
 struct QGeom {
-    static constexpr int G = B / kEPT;                 // threads per block-group
+    static constexpr int CW = WIDE ? 8 : 4;
+    static constexpr int EPT = BF16 ? 32 : 16;
+    static constexpr int NCH = EPT / CW;
+    static constexpr int G = B / EPT;                  // threads per block-group
     static constexpr int kGroups = kQThreads / G;      // block-groups per CTA
     static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
     static constexpr size_t kSmem = sizeof(CodeSmem) + sizeof(float) * kGroups * 2 * kGroupWarps;
+    static_assert(G >= 1 && kQThreads % G == 0 && (!WIDE || BF16), "group geometry");
 };
-template <bool BF16, bool FULL>
-__device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, float (&v)[4])
+
+template <bool BF16, int CW, bool FULL>
+__device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, float (&v)[CW])
 {
-    if (FULL || e + 4 <= n) {
-        if (BF16) {
-            uint2 w = ld_stream_u2(static_cast<const uint16_t*>(A) + e);
+    if (FULL || e + CW <= n) {
+        if constexpr (BF16 && CW == 8) {
+            const uint4 w = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(A) + e));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                v[2 * i] = bf16lo_to_f32(ws[i]);
+                v[2 * i + 1] = bf16hi_to_f32(ws[i]);
+            }
+        } else if constexpr (BF16) {
+            const uint2 w = ld_stream_u2(static_cast<const uint16_t*>(A) + e);
             v[0] = bf16lo_to_f32(w.x);
             v[1] = bf16hi_to_f32(w.x);
             v[2] = bf16lo_to_f32(w.y);
             v[3] = bf16hi_to_f32(w.y);
         } else {
-            float4 f = ld_stream_f4(static_cast<const float*>(A) + e);
+            const float4 f = ld_stream_f4(static_cast<const float*>(A) + e);
             v[0] = f.x;
             v[1] = f.y;
             v[2] = f.z;
@@ -51,7 +68,7 @@ __device__ __forceinline__ void load_chunk(const void* A, int64_t e, int64_t n, 
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
+        for (int i = 0; i < CW; i++) {
             float x = 0.0f;
             if (e + i < n) {
                 if (BF16)
@@ -85,78 +102,97 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
     return true;
 }
 
+// The codes of 4 consecutive elements, byte i = code of element i.
+template <int MODE, bool FAST>
+__device__ __forceinline__ uint32_t codes4(const CodeSmem& cs, const BlockScale& sc, const float* x)
+{
+    float2 x0 = make_float2(x[0], x[1]), x1 = make_float2(x[2], x[3]);
+    if (FAST) {
+        const float2 r = make_float2(sc.r, sc.r), na = make_float2(sc.na, sc.na);
+        x0 = div2_rcp(x0, r, na);
+        x1 = div2_rcp(x1, r, na);
+    } else {
+        x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
+        x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
+    }
+    return pack_top_bytes(nearest_code_word<MODE>(cs, x0.x), nearest_code_word<MODE>(cs, x0.y),
+                          nearest_code_word<MODE>(cs, x1.x), nearest_code_word<MODE>(cs, x1.y));
+}
+
+// Two 4-bit codes per byte, the even element in the high nibble: bytes 0 and 2 of
+// (word << 4) | (word >> 8) hold (c0 << 4 | c1) and (c2 << 4 | c3) for a word of codes below 16.
+__device__ __forceinline__ uint32_t nibble_pairs(uint32_t word) { return (word << 4) | (word >> 8); }
+
 // Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division; FULL:
 // the block lies entirely inside the tensor, so no element needs a bounds check).
-template <int B, int K, int MODE, bool FAST, bool FULL>
-__device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockScale& sc, const float (&v)[4][4],
+template <int B, bool BF16, bool WIDE, int K, int MODE, bool FAST, bool FULL>
+__device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockScale& sc,
+                                               const float (&v)[QGeom<B, BF16, WIDE>::NCH][QGeom<B, BF16, WIDE>::CW],
                                                int64_t base, int tg, int64_t n, uint8_t* __restrict__ out)
 {
-    constexpr int G = QGeom<B>::G;
-    const float2 r = make_float2(sc.r, sc.r), na = make_float2(sc.na, sc.na);
+    using Geo = QGeom<B, BF16, WIDE>;
+    constexpr int G = Geo::G, CW = Geo::CW;
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-        const int64_t e = base + 4 * (j * G + tg);
+    for (int j = 0; j < Geo::NCH; j++) {
+        const int64_t e = base + CW * (j * G + tg);
         if (!FULL && e >= n) continue;
-        float2 x0 = make_float2(v[j][0], v[j][1]), x1 = make_float2(v[j][2], v[j][3]);
-        if (FAST) {
-            x0 = div2_rcp(x0, r, na);
-            x1 = div2_rcp(x1, r, na);
-        } else {
-            x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
-            x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
-        }
-        const uint32_t w0 = nearest_code_word<MODE>(cs, x0.x), w1 = nearest_code_word<MODE>(cs, x0.y);
-        const uint32_t w2 = nearest_code_word<MODE>(cs, x1.x), w3 = nearest_code_word<MODE>(cs, x1.y);
-        const uint32_t word = pack_top_bytes(w0, w1, w2, w3);  // byte i = code of element e + i
-        if constexpr (K == 256) {
-            if (FULL || e + 4 <= n) {
-                st_stream_u32(out + e, word);
+        uint32_t word[CW / 4];
+#pragma unroll
+        for (int h = 0; h < CW / 4; h++) word[h] = codes4<MODE, FAST>(cs, sc, &v[j][4 * h]);
+        if (FULL || e + CW <= n) {
+            if constexpr (K == 256 && CW == 8) {
+                st_stream_u2(out + e, make_uint2(word[0], word[1]));
+            } else if constexpr (K == 256) {
+                st_stream_u32(out + e, word[0]);
+            } else if constexpr (CW == 8) {
+                st_stream_u32(out + (e >> 1), __byte_perm(nibble_pairs(word[0]), nibble_pairs(word[1]), 0x6420u));
             } else {
-                out[e] = (uint8_t)word;
-                if (e + 1 < n) out[e + 1] = (uint8_t)(word >> 8);
-                if (e + 2 < n) out[e + 2] = (uint8_t)(word >> 16);
+                *reinterpret_cast<uint16_t*>(out + (e >> 1)) = (uint16_t)__byte_perm(nibble_pairs(word[0]), 0u, 0x4420u);
             }
-        } else {  // two 4-bit codes per byte, even element in the high nibble
-            // (word << 4) | (word >> 8): byte 0 = q0 << 4 | q1 and byte 2 = q2 << 4 | q3 (codes < 16)
-            const uint32_t u = (word << 4) | (word >> 8);
-            uint8_t* o = out + (e >> 1);
-            if (FULL || e + 4 <= n) {
-                *reinterpret_cast<uint16_t*>(o) = (uint16_t)__byte_perm(u, 0u, 0x4420u);
-            } else {  // the low nibble past the end stays 0
-                const uint32_t keep = e + 1 < n ? 0xffu : 0xf0u;
-                o[0] = (uint8_t)(u & keep);
-                if (e + 2 < n) o[1] = (uint8_t)((u >> 16) & (e + 3 < n ? 0xffu : 0xf0u));
+        } else {  // the tensor's last, partial chunk: element by element
+#pragma unroll
+            for (int i = 0; i < CW; i++) {
+                if (e + i >= n) break;
+                const uint32_t c = (word[i >> 2] >> (8 * (i & 3))) & 0xffu;
+                if constexpr (K == 256) {
+                    out[e + i] = (uint8_t)c;
+                } else if ((i & 1) == 0) {  // the high nibble; a missing partner leaves the low one 0
+                    const uint32_t c1 = e + i + 1 < n ? (word[(i + 1) >> 2] >> (8 * ((i + 1) & 3))) & 0xffu : 0u;
+                    out[(e + i) >> 1] = (uint8_t)((c << 4) | c1);
+                }
             }
         }
     }
 }
 
 // One block: loads, block absmax over the group, normalise, search, store.
-template <int B, bool BF16, int K, int MODE, bool CENTER, bool FULL>
+// CENTER: quantize A[i] - off (one binary32 subtraction; fp32 input), the centred block scales of
+// nested quantization.
+template <int B, bool BF16, bool WIDE, int K, int MODE, bool CENTER, bool FULL>
 __device__ __forceinline__ void quantize_block(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
                                                float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
                                                unsigned* flags, float off, int64_t b, int gi, int tg, int lane,
                                                unsigned gmask, int& parity)
 {
-    constexpr int G = QGeom<B>::G;
+    using Geo = QGeom<B, BF16, WIDE>;
+    constexpr int G = Geo::G, CW = Geo::CW, NCH = Geo::NCH;
     const int64_t base = b * B;
-    float v[4][4];
+    float v[NCH][CW];
 #pragma unroll
-    for (int j = 0; j < 4; j++) load_chunk<BF16, FULL>(A, base + 4 * (j * G + tg), n, v[j]);
+    for (int j = 0; j < NCH; j++) load_chunk<BF16, CW, FULL>(A, base + CW * (j * G + tg), n, v[j]);
     if constexpr (CENTER) {
 #pragma unroll
-        for (int j = 0; j < 4; j++)
+        for (int j = 0; j < NCH; j++)
 #pragma unroll
-            for (int i = 0; i < 4; i++)
-                if (FULL || base + 4 * (j * G + tg) + i < n) v[j][i] = __fsub_rn(v[j][i], off);
+            for (int i = 0; i < CW; i++)
+                if (FULL || base + CW * (j * G + tg) + i < n) v[j][i] = __fsub_rn(v[j][i], off);
     }
 
     float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-        m = max3_abs_nan(m, v[j][0], v[j][1]);
-        m = max3_abs_nan(m, v[j][2], v[j][3]);
-    }
+    for (int j = 0; j < NCH; j++)
+#pragma unroll
+        for (int i = 0; i < CW; i += 2) m = max3_abs_nan(m, v[j][i], v[j][i + 1]);
 
     if constexpr (G <= 32) {
         m = group_max_nan<G>(m, gmask);
@@ -176,19 +212,17 @@ __device__ __forceinline__ void quantize_block(const CodeSmem& cs, bool fast, co
     }
     const BlockScale sc = make_scale(m, fast);
     if (sc.fast)
-        quantize_store<B, K, MODE, true, FULL>(cs, sc, v, base, tg, n, out);
+        quantize_store<B, BF16, WIDE, K, MODE, true, FULL>(cs, sc, v, base, tg, n, out);
     else
-        quantize_store<B, K, MODE, false, FULL>(cs, sc, v, base, tg, n, out);
+        quantize_store<B, BF16, WIDE, K, MODE, false, FULL>(cs, sc, v, base, tg, n, out);
 }
 
-// CENTER: quantize A[i] - *center (one binary32 subtraction; fp32 input), the centred block
-// scales of nested quantization.
-template <int B, bool BF16, int K, int MODE, bool CENTER>
+template <int B, bool BF16, bool WIDE, int K, int MODE, bool CENTER>
 __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, const void* __restrict__ A, int64_t n,
                                               float* __restrict__ absmax, uint8_t* __restrict__ out, float* red,
                                               unsigned* flags, const float* __restrict__ center)
 {
-    using Geo = QGeom<B>;
+    using Geo = QGeom<B, BF16, WIDE>;
     constexpr int G = Geo::G;
     const int gi = threadIdx.x / G;
     const int tg = threadIdx.x % G;
@@ -200,15 +234,15 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
 
     for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb; b += (int64_t)gridDim.x * Geo::kGroups) {
         if ((b + 1) * B <= n)  // group-uniform: every thread of the group holds the same block
-            quantize_block<B, BF16, K, MODE, CENTER, true>(cs, fast, A, n, absmax, out, red, flags, off, b, gi, tg,
-                                                           lane, gmask, parity);
+            quantize_block<B, BF16, WIDE, K, MODE, CENTER, true>(cs, fast, A, n, absmax, out, red, flags, off, b, gi,
+                                                                 tg, lane, gmask, parity);
         else
-            quantize_block<B, BF16, K, MODE, CENTER, false>(cs, fast, A, n, absmax, out, red, flags, off, b, gi, tg,
-                                                            lane, gmask, parity);
+            quantize_block<B, BF16, WIDE, K, MODE, CENTER, false>(cs, fast, A, n, absmax, out, red, flags, off, b, gi,
+                                                                  tg, lane, gmask, parity);
     }
 }
 
-template <int B, bool BF16, int K, bool CENTER>
+template <int B, bool BF16, bool WIDE, int K, bool CENTER>
 __global__ void __launch_bounds__(kQThreads, 2)
 quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int64_t n,
                 float* __restrict__ absmax, uint8_t* __restrict__ out, unsigned* flags,
@@ -220,11 +254,11 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     bool fast, general;
     if (!stage_one_code(cs, code, K, true, fast, general, flags)) return;
     if (general)
-        quantize_loop<B, BF16, K, kSearchGeneral, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
+        quantize_loop<B, BF16, WIDE, K, kSearchGeneral, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
     else if (cs.code[0] >= 0.0f)  // every code >= 0
-        quantize_loop<B, BF16, K, kSearchNonNeg, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
+        quantize_loop<B, BF16, WIDE, K, kSearchNonNeg, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
     else
-        quantize_loop<B, BF16, K, kSearchSigned, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
+        quantize_loop<B, BF16, WIDE, K, kSearchSigned, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
 }
 
 // Dequantize: a lane's unit is 16 bytes of output (8 bf16 or 4 fp32 elements, always inside one
@@ -388,15 +422,15 @@ bnbq_status persistent_grid(Kern kern, int threads, size_t smem, int64_t work_un
     return BNBQ_OK;
 }
 
-template <int B, bool BF16, int K, bool CENTER = false>
+template <int B, bool BF16, bool WIDE, int K, bool CENTER = false>
 bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax, uint8_t* out,
                      cudaStream_t s, const float* center = nullptr)
 {
-    using Geo = QGeom<B>;
+    using Geo = QGeom<B, BF16, WIDE>;
     unsigned* flags = nullptr;
     bnbq_status st = device_flag_ptr(&flags);
     if (st != BNBQ_OK) return st;
-    auto kern = quantize_kernel<B, BF16, K, CENTER>;
+    auto kern = quantize_kernel<B, BF16, WIDE, K, CENTER>;
     // The kernel's shared-memory limit, set once per device (for this instantiation).
     constexpr int kDevs = 64;
     static std::mutex mu;
@@ -420,12 +454,19 @@ bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax,
     return cuda_status(cudaGetLastError(), "quantize_kernel launch");
 }
 
+// bf16 input 16-byte aligned, with codes aligned for 8 (8-bit) or 4 (4-bit) bytes per store:
+// 8-element chunks; otherwise 4-element chunks.
 template <int B, bool BF16>
 bnbq_status launch_q_k(const float* code, int K, const void* A, int64_t n, float* absmax,
                        uint8_t* out, cudaStream_t s)
 {
-    return K == 256 ? launch_q<B, BF16, 256>(code, A, n, absmax, out, s)
-                    : launch_q<B, BF16, 16>(code, A, n, absmax, out, s);
+    const bool wide = BF16 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0 &&
+                      (reinterpret_cast<uintptr_t>(out) & (K == 256 ? 7u : 3u)) == 0;
+    if (wide)
+        return K == 256 ? launch_q<B, true, true, 256>(code, A, n, absmax, out, s)
+                        : launch_q<B, true, true, 16>(code, A, n, absmax, out, s);
+    return K == 256 ? launch_q<B, BF16, false, 256>(code, A, n, absmax, out, s)
+                    : launch_q<B, BF16, false, 16>(code, A, n, absmax, out, s);
 }
 
 template <int B>
@@ -472,7 +513,7 @@ bnbq_status launch_quantize(const float* code, int K, const void* A, bnbq_dtype 
 bnbq_status launch_quantize_centred(const float* code2, const float* a, int64_t nb, const float* center,
                                     float* absmax2, uint8_t* qabs, cudaStream_t s)
 {
-    return launch_q<kNestBlock, false, 256, true>(code2, a, nb, absmax2, qabs, s, center);
+    return launch_q<kNestBlock, false, false, 256, true>(code2, a, nb, absmax2, qabs, s, center);
 }
 
 bnbq_status launch_dequantize_nested(const float* code, int K, const uint8_t* q, const uint8_t* qabs,

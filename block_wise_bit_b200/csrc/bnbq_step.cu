@@ -254,6 +254,14 @@ __device__ __forceinline__ void store_q4(uint8_t* q, int64_t e, int64_t n, uint3
 
 __device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return __byte_perm(w, 0u, 0x4440u + (uint32_t)i); }
 
+// code[byte i of w], with the byte's table offset 4 * byte formed by one shift and one mask (i is
+// a compile-time constant in the unrolled loops).
+__device__ __forceinline__ float code_at(const float* code, uint32_t w, int i)
+{
+    const uint32_t off = (i == 0 ? (w << 2) : (w >> (8 * i - 2))) & 0x3fcu;
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(code) + off);
+}
+
 // Group-wide max of (x, y) over the G threads of one block-group, in two halves so that work
 // independent of the result can run between them: group_max_publish reduces inside each warp
 // (and, for groups of several warps, stores the warp's maxima to shared memory, double-buffered
@@ -445,10 +453,10 @@ __device__ __forceinline__ void block8(const Cur& c, int64_t lb, const StepScala
         float2 ph[2] = {make_float2(pv[j].x, pv[j].y), make_float2(pv[j].z, pv[j].w)};
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            float2 m = mul2(make_float2(code1[byte_of(w1[j], 2 * h)], code1[byte_of(w1[j], 2 * h + 1)]), a1p);
+            float2 m = mul2(make_float2(code_at(code1, w1[j], 2 * h), code_at(code1, w1[j], 2 * h + 1)), a1p);
             float2 v = make_float2(0.0f, 0.0f);
             if constexpr (TWO)
-                v = mul2(make_float2(code2[byte_of(w2[j], 2 * h)], code2[byte_of(w2[j], 2 * h + 1)]), a2p);
+                v = mul2(make_float2(code_at(code2, w2[j], 2 * h), code_at(code2, w2[j], 2 * h + 1)), a2p);
             states2<OPT>(sc, kp, ph[h], gv[j].half(h), m, v);
             if (!FULL) {  // elements past the end do not count towards the block scale
                 if (e + 2 * h >= n) { m.x = 0.0f; v.x = 0.0f; }

@@ -117,6 +117,40 @@ def test_small_and_ragged(n, code_name):
         _check_full(code, x, B)
 
 
+@pytest.mark.parametrize("n", [1, 5, 7, 8, 9, 31, 33, 63, 64, 65, 127, 129, 2049, 65 * 64 + 3])
+@pytest.mark.parametrize("code_name", ["signed", "nf4"])
+def test_small_and_ragged_bf16(n, code_name):
+    """bf16 input, whose full blocks take 8-element chunks: ragged tails inside a chunk and a
+    block, for the 4-bit weight blocksize and the optimizer-state ones."""
+    code = _codes()[code_name]
+    x = sweep_input(n, torch.bfloat16, f"ragged-bf16-{n}")
+    for B in (64, 256, 2048):
+        _check_full(code, x, B)
+
+
+@pytest.mark.parametrize("code_name", ["signed", "nf4"])
+def test_bf16_input_and_codes_at_narrow_alignment(code_name):
+    """bf16 input only 8-byte aligned and codes only as aligned as the interface asks (4 bytes for
+    8-bit codes, 2 for 4-bit): the kernel falls back to 4-element chunks; results as the oracle's."""
+    code = _codes()[code_name]
+    n, B = 64 * 1000 + 37, 64
+    K = code.numel()
+    xf = sweep_input(n + 4, torch.bfloat16, "narrow")
+    x = xf[4:]                                  # 8 bytes past a 16-byte boundary
+    assert x.data_ptr() % 16 == 8
+    nq = n if K == 256 else (n + 1) // 2
+    step = 4 if K == 256 else 2
+    qf = torch.full((nq + step + 64,), 0xA5, dtype=torch.uint8, device=DEV)
+    q = qf[step:step + nq]                      # 4 (8-bit) or 2 (4-bit) bytes past an 8-byte boundary
+    a = torch.empty((n + B - 1) // B, dtype=torch.float32, device=DEV)
+    bq.bnbq_quantize_blockwise(code.to(DEV), x, B, absmax=a, out=q)
+    torch.cuda.synchronize()
+    assert bool((qf[:step] == 0xA5).all()) and bool((qf[step + nq:] == 0xA5).all()), "write outside the codes"
+    a_or, q_or = oracle.quantize_blockwise(code.numpy(), parity.to_np(x), B)
+    np.testing.assert_array_equal(parity.to_np(a).view(np.uint32), a_or.view(np.uint32))
+    np.testing.assert_array_equal(parity.to_np(q), q_or)
+
+
 def test_empty_is_noop():
     code = _codes()["signed"].to(DEV)
     x = torch.empty(0, device=DEV)
