@@ -102,9 +102,19 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
     return true;
 }
 
-// The codes of 4 consecutive elements, byte i = code of element i.
+// Nearest-code word of a normalised value in the kernel's search mode (code in the top byte).
+template <int MODE>
+__device__ __forceinline__ uint32_t code_word(const CodeSmem& cs, float x)
+{
+    if constexpr (MODE == kSearchPrefix12)
+        return nearest_code_word12(cs.table, x);
+    else
+        return nearest_code_word<MODE>(cs, x);
+}
+
+// The four nearest-code words of 4 consecutive elements.
 template <int MODE, bool FAST>
-__device__ __forceinline__ uint32_t codes4(const CodeSmem& cs, const BlockScale& sc, const float* x)
+__device__ __forceinline__ void words4(const CodeSmem& cs, const BlockScale& sc, const float* x, uint32_t (&w)[4])
 {
     float2 x0 = make_float2(x[0], x[1]), x1 = make_float2(x[2], x[3]);
     if (FAST) {
@@ -115,13 +125,32 @@ __device__ __forceinline__ uint32_t codes4(const CodeSmem& cs, const BlockScale&
         x0 = make_float2(__fdiv_rn(x0.x, sc.a), __fdiv_rn(x0.y, sc.a));
         x1 = make_float2(__fdiv_rn(x1.x, sc.a), __fdiv_rn(x1.y, sc.a));
     }
-    return pack_top_bytes(nearest_code_word<MODE>(cs, x0.x), nearest_code_word<MODE>(cs, x0.y),
-                          nearest_code_word<MODE>(cs, x1.x), nearest_code_word<MODE>(cs, x1.y));
+    w[0] = code_word<MODE>(cs, x0.x);
+    w[1] = code_word<MODE>(cs, x0.y);
+    w[2] = code_word<MODE>(cs, x1.x);
+    w[3] = code_word<MODE>(cs, x1.y);
 }
 
-// Two 4-bit codes per byte, the even element in the high nibble: bytes 0 and 2 of
-// (word << 4) | (word >> 8) hold (c0 << 4 | c1) and (c2 << 4 | c3) for a word of codes below 16.
-__device__ __forceinline__ uint32_t nibble_pairs(uint32_t word) { return (word << 4) | (word >> 8); }
+// The codes of 4 consecutive elements, byte i = code of element i.
+template <int MODE, bool FAST>
+__device__ __forceinline__ uint32_t codes4(const CodeSmem& cs, const BlockScale& sc, const float* x)
+{
+    uint32_t w[4];
+    words4<MODE, FAST>(cs, sc, x, w);
+    return pack_top_bytes(w[0], w[1], w[2], w[3]);
+}
+
+// The 4-bit codes of 4 consecutive elements packed two per byte (even element in the high nibble)
+// in the low 16 bits, formed with integer multiply-adds (codes below 16).
+template <int MODE, bool FAST>
+__device__ __forceinline__ uint32_t nibbles4(const CodeSmem& cs, const BlockScale& sc, const float* x)
+{
+    uint32_t w[4];
+    words4<MODE, FAST>(cs, sc, x, w);
+    const uint32_t b0 = (w[0] >> 24) * 16u + (w[1] >> 24);
+    const uint32_t b1 = (w[2] >> 24) * 16u + (w[3] >> 24);
+    return b1 * 256u + b0;
+}
 
 // Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division; FULL:
 // the block lies entirely inside the tensor, so no element needs a bounds check).
@@ -136,19 +165,24 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
     for (int j = 0; j < Geo::NCH; j++) {
         const int64_t e = base + CW * (j * G + tg);
         if (!FULL && e >= n) continue;
+        if constexpr (K == 16) {
+            if (FULL || e + CW <= n) {
+                if constexpr (CW == 8)
+                    st_stream_u32(out + (e >> 1), nibbles4<MODE, FAST>(cs, sc, &v[j][4]) * 65536u +
+                                                      nibbles4<MODE, FAST>(cs, sc, &v[j][0]));
+                else
+                    *reinterpret_cast<uint16_t*>(out + (e >> 1)) = (uint16_t)nibbles4<MODE, FAST>(cs, sc, &v[j][0]);
+                continue;
+            }
+        }
         uint32_t word[CW / 4];
 #pragma unroll
         for (int h = 0; h < CW / 4; h++) word[h] = codes4<MODE, FAST>(cs, sc, &v[j][4 * h]);
         if (FULL || e + CW <= n) {
-            if constexpr (K == 256 && CW == 8) {
+            if constexpr (K == 256 && CW == 8)
                 st_stream_u2(out + e, make_uint2(word[0], word[1]));
-            } else if constexpr (K == 256) {
+            else
                 st_stream_u32(out + e, word[0]);
-            } else if constexpr (CW == 8) {
-                st_stream_u32(out + (e >> 1), __byte_perm(nibble_pairs(word[0]), nibble_pairs(word[1]), 0x6420u));
-            } else {
-                *reinterpret_cast<uint16_t*>(out + (e >> 1)) = (uint16_t)__byte_perm(nibble_pairs(word[0]), 0u, 0x4420u);
-            }
         } else {  // the tensor's last, partial chunk: element by element
 #pragma unroll
             for (int i = 0; i < CW; i++) {
@@ -252,7 +286,19 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     CodeSmem& cs = *reinterpret_cast<CodeSmem*>(smem_raw);
     float* red = reinterpret_cast<float*>(smem_raw + sizeof(CodeSmem));
     bool fast, general;
-    if (!stage_one_code(cs, code, K, true, fast, general, flags)) return;
+    if constexpr (K == 16) {
+        // 16 codes: the 12-bit-prefix table when no bucket of it holds two midpoints
+        if (!stage_one_code(cs, code, K, false, fast, general, flags)) return;
+        if (!__syncthreads_or(build_table12(cs.table, cs.mid, K))) {
+            __syncthreads();
+            quantize_loop<B, BF16, WIDE, K, kSearchPrefix12, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
+            return;
+        }
+        __syncthreads();
+        general = __syncthreads_or(stage_code_pass3(cs, K));
+    } else if (!stage_one_code(cs, code, K, true, fast, general, flags)) {
+        return;
+    }
     if (general)
         quantize_loop<B, BF16, WIDE, K, kSearchGeneral, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
     else if (cs.code[0] >= 0.0f)  // every code >= 0
@@ -261,12 +307,20 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
         quantize_loop<B, BF16, WIDE, K, kSearchSigned, CENTER>(cs, fast, A, n, absmax, out, red, flags, center);
 }
 
+// code[nibble i of w] of a 16-entry codebook (nibble 0 = bits 0..3), its table offset formed by one
+// shift and one mask.  The 16 codes sit in 16 different shared-memory banks, so these lookups
+// never conflict (a table of code pairs indexed by the whole byte, read 8 bytes at a time,
+// conflicted about three times per access).
+__device__ __forceinline__ float code16_at(const float* code, uint32_t w, int i)
+{
+    const uint32_t off = (i == 0 ? (w << 2) : (w >> (4 * i - 2))) & 0x3cu;
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(code) + off);
+}
+
 // Dequantize: a lane's unit is 16 bytes of output (8 bf16 or 4 fp32 elements, always inside one
 // block); consecutive lanes take consecutive units, so every load and store instruction of a warp
-// covers one contiguous range.  8-bit codes: one
-// table lookup per element, one packed product per pair.  4-bit codes: a 256-entry table of code
-// pairs indexed by the whole byte (high nibble = the even element): one shared load and one
-// packed product per two elements.
+// covers one contiguous range.  One table lookup per element (for 4-bit codes the high nibble of
+// a byte is the even element) and one packed product per pair.
 // NESTED: the block scales are rebuilt from their nested quantization,
 // A_b = code2[qabs_b] * absmax2[b / 256] + *center (two roundings), instead of read from absmax.
 struct NestedScales {
@@ -301,15 +355,12 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
     using Wd = DqWords<K, UE>;
     __shared__ float code_s[NESTED ? 2 : 1][256];
     __shared__ float mid_s[NESTED ? 2 : 1][256];
-    __shared__ float2 pair_s[K == 16 ? 256 : 1];  // 4-bit: byte -> (code[hi nibble], code[lo nibble])
     stage_codes(code_s[0], code, K);
     if constexpr (NESTED) stage_codes(code_s[NESTED ? 1 : 0], ns.code2, 256);
     __syncthreads();
     bool bad = false, tiny = false;
     stage_midpoints(code_s[0], mid_s[0], K, bad, tiny);
     if constexpr (NESTED) stage_midpoints(code_s[NESTED ? 1 : 0], mid_s[NESTED ? 1 : 0], 256, bad, tiny);
-    if constexpr (K == 16)
-        for (int b = threadIdx.x; b < 256; b += blockDim.x) pair_s[b] = make_float2(code_s[0][b >> 4], code_s[0][b & 15]);
     if (__syncthreads_or(bad)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags, kFlagBadCode);
         return;
@@ -375,8 +426,9 @@ dequantize_kernel(const float* __restrict__ code, const uint8_t* __restrict__ q,
                     const uint32_t b0 = 2u * (h & 1);
                     y[h] = mul2(make_float2(code_s[0][__byte_perm(wd, 0u, 0x4440u + b0)],
                                             code_s[0][__byte_perm(wd, 0u, 0x4441u + b0)]), ap);
-                } else {
-                    y[h] = mul2(pair_s[__byte_perm(w[j][0], 0u, 0x4440u + h)], ap);
+                } else {  // byte h holds elements 2h (high nibble) and 2h+1 (low nibble)
+                    y[h] = mul2(make_float2(code16_at(code_s[0], w[j][0], 2 * h + 1),
+                                            code16_at(code_s[0], w[j][0], 2 * h)), ap);
                 }
             }
             if (e + UE <= n) {

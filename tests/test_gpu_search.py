@@ -35,3 +35,5 @@ def test_search_exhaustive(checker, tmp_path, kind):
     out = subprocess.run([str(checker), str(f), str(code.size)], capture_output=True, text=True, timeout=600)
     assert out.returncode == 0 and "result ok" in out.stdout, out.stdout + out.stderr
     assert "midpoints equal" in out.stdout and "mode general status no error mismatches 0" in out.stdout
+    if code.size == 16:  # the quantize kernel's search for 16 codes
+        assert "mode prefix12 status no error mismatches 0" in out.stdout, out.stdout
