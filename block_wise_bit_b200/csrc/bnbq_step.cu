@@ -562,18 +562,6 @@ __device__ __forceinline__ void block32(const Cur& c, int64_t lb, const StepScal
     }
 }
 
-#ifndef BNBQ_STEP_PREFETCH
-#define BNBQ_STEP_PREFETCH 0  // blocks ahead whose streams are prefetched into L2 (0: none)
-#endif
-// Bulk prefetch of [p, p + bytes) into L2, widened to 16-byte boundaries (the caller keeps the
-// widened range inside the tensor).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
-{
-    const uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~(uintptr_t)15;
-    const uintptr_t e = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~(uintptr_t)15;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"((uint32_t)(e - a)) : "memory");
-}
-
 template <int OPT, int B, int M1, int M2>
 __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, int ntensors, int total_blocks,
                                           const StepScalars& sc, const StepSmem<OptTraits<OPT>::kCodes>& cs,
@@ -599,21 +587,6 @@ __device__ __forceinline__ void step_loop(const StepDesc* __restrict__ table, in
         Cur c;
         load_cur(c, table, cur, ntensors);
         const int64_t lb = (int64_t)(b - c.first);
-        if (BNBQ_STEP_PREFETCH > 0 && tg == 0 && (c.flags & kDescState8)) {
-            // the group's block BNBQ_STEP_PREFETCH strides ahead, if it is an inner block of this
-            // tensor (so the 16-byte widening stays inside the tensor)
-            const int bn = b + BNBQ_STEP_PREFETCH * gridDim.x * Geo::kGroups;
-            if (bn < next_first) {
-                const int64_t ln = (int64_t)(bn - c.first);
-                if (ln >= 1 && (ln + 2) * B <= c.n) {
-                    const uint32_t gsz = (c.flags & kDescGBf16) ? 2u : 4u;
-                    prefetch_l2(c.p + ln * B, 4u * B);
-                    prefetch_l2(static_cast<const char*>(c.g) + ln * B * gsz, gsz * B);
-                    prefetch_l2(c.q1 + ln * B, B);
-                    if constexpr (OptTraits<OPT>::kTwoStates) prefetch_l2(c.q2 + ln * B, B);
-                }
-            }
-        }
         if (c.flags & kDescState8) {
             const bool full = (lb + 1) * B <= c.n;
             if (c.flags & kDescGBf16) {
