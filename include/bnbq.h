@@ -14,6 +14,9 @@
  * Conventions for every entry point:
  *  - Pointers named as device memory must point to memory of the current CUDA device; host
  *    structs are read before the call returns and not kept.  The caller owns every buffer.
+ *    Codebook pointers are checked before anything is launched: one that is not device (or
+ *    managed) memory of the current device, or whose codes would run past the end of its
+ *    allocation as the driver reports it, returns BNBQ_EINVAL.
  *  - Work is enqueued on `stream` (NULL = the legacy default stream) and is asynchronous with
  *    respect to the host.  Argument checks are synchronous: a non-OK status means nothing was
  *    enqueued.  BNBQ_ECUDA means a CUDA call failed; the CUDA error text is in bnbq_last_error().
