@@ -103,18 +103,23 @@ def quant_point(point, steps, warmup, seed_tag):
     alg_q = n * esz + qbytes + 4 * nb
     alg_dq = qbytes + 4 * nb + n * esz
     stream = torch.cuda.current_stream(dev)
-    code2 = None
+    code2 = nest_bufs = None
     if nested:  # nest: read the scales twice (mean, quantize), write codes + second-level scales
         code2 = bq.bnbq_codebook("dynamic_signed").to(dev)
         nb2 = (nb + 255) // 256
         alg_q += 8 * nb + nb + 4 * nb2
         alg_dq = qbytes + nb + 4 * nb2 + n * esz
+        nest_bufs = dict(qabs=torch.empty(nb, dtype=torch.uint8, device=dev),
+                         absmax2=torch.empty(nb2, dtype=torch.float32, device=dev),
+                         offset=torch.empty(1, dtype=torch.float32, device=dev),
+                         workspace=torch.empty(max(1, bq.lib().bnbq_nested_workspace_bytes(nb)), dtype=torch.uint8,
+                                               device=dev))
     # each call's bytes well above L2, or L2 is overwritten before every timed call
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if min(alg_q, alg_dq) < 2 * L2_BYTES else None
 
     def quantize():
         bq.bnbq_quantize_blockwise(code, x, B, absmax=absmax, out=q)
-        return bq.bnbq_quantize_absmax_nested(code2, absmax) if nested else None
+        return bq.bnbq_quantize_absmax_nested(code2, absmax, **nest_bufs) if nested else None
 
     def dequantize(nest):
         if nested:

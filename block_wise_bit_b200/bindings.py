@@ -203,20 +203,27 @@ def bnbq_dequantize_blockwise(code: torch.Tensor, q: torch.Tensor, absmax: torch
 NEST_BLOCK = 256
 
 
-def bnbq_quantize_absmax_nested(code2: torch.Tensor, absmax: torch.Tensor, stream=None):
+def bnbq_quantize_absmax_nested(code2: torch.Tensor, absmax: torch.Tensor, stream=None,
+                                qabs: Optional[torch.Tensor] = None, absmax2: Optional[torch.Tensor] = None,
+                                offset: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
     """Nested quantization of a block-scale array: returns (qabs uint8[nb], absmax2 float32
-    [ceil(nb/256)], offset float32[1]), all on absmax's device.  The workspace is a torch
-    allocation made here."""
+    [ceil(nb/256)], offset float32[1]), all on absmax's device.  Outputs and the workspace
+    (``bnbq_nested_workspace_bytes(nb)`` bytes) may be passed in to reuse them; missing ones are
+    torch allocations made here."""
     nb = absmax.numel()
     dev = absmax.device
-    qabs = torch.empty(nb, dtype=torch.uint8, device=dev)
-    absmax2 = torch.empty((nb + NEST_BLOCK - 1) // NEST_BLOCK, dtype=torch.float32, device=dev)
-    offset = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, lib().bnbq_nested_workspace_bytes(nb)), dtype=torch.uint8, device=dev)
+    if qabs is None:
+        qabs = torch.empty(nb, dtype=torch.uint8, device=dev)
+    if absmax2 is None:
+        absmax2 = torch.empty((nb + NEST_BLOCK - 1) // NEST_BLOCK, dtype=torch.float32, device=dev)
+    if offset is None:
+        offset = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(1, lib().bnbq_nested_workspace_bytes(nb)), dtype=torch.uint8, device=dev)
     _check(lib().bnbq_quantize_absmax_nested(_dev(absmax, "absmax") if nb else None, nb, _dev(code2, "code2"),
                                              _dev(qabs, "qabs") if nb else None,
                                              _dev(absmax2, "absmax2") if nb else None, _dev(offset, "offset"),
-                                             _dev(ws, "workspace"), _stream(stream)))
+                                             _dev(workspace, "workspace"), _stream(stream)))
     return qabs, absmax2, offset
 
 

@@ -45,7 +45,6 @@ __device__ __forceinline__ int max_over_block(int v)
 // of U's that a double holds exactly.  Otherwise (a wider spread, or a NaN or infinity) one thread
 // adds in index order.
 constexpr int kSumThreads = 256;
-constexpr int kPerThread = kNestChunk / kSumThreads;  // 16 consecutive values per thread
 
 __device__ __forceinline__ int ulp_exponent(float x)  // biased exponent of x's ulp; 1 for subnormals
 {
@@ -63,9 +62,10 @@ absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ 
     for (int i = threadIdx.x; i < len; i += blockDim.x) chunk[i] = __ldg(a + start + i);
     __syncthreads();
     // ulp exponent range of the non-zero values (a NaN or infinity forces the ordered sum)
+    // (threads take every kSumThreads-th value: consecutive threads read consecutive words, so the
+    // shared-memory reads never conflict; the exact sum below does not depend on the order)
     int emin = 255, emax = 0;
-    const int i0 = threadIdx.x * kPerThread;
-    for (int i = i0; i < i0 + kPerThread && i < len; i++) {
+    for (int i = threadIdx.x; i < len; i += kSumThreads) {
         const float x = chunk[i];
         if (x == 0.0f) continue;
         const int e = ulp_exponent(x);
@@ -77,7 +77,7 @@ absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ 
     const bool exact = emax - emin <= 17;
     if (exact) {  // every order gives the same (exact) sum
         double s = 0.0;
-        for (int i = i0; i < i0 + kPerThread && i < len; i++) s = __dadd_rn(s, (double)chunk[i]);
+        for (int i = threadIdx.x; i < len; i += kSumThreads) s = __dadd_rn(s, (double)chunk[i]);
         for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
         if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
         __syncthreads();
@@ -94,13 +94,24 @@ absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ 
     work[blockIdx.x] = s;
 }
 
-__global__ void __launch_bounds__(32)
+// The chunk sums in index order: the CTA stages them in shared memory with coalesced loads, a
+// tile at a time, and one thread adds them up (the order is part of the definition).
+constexpr int kFinishTile = 2048;
+
+__global__ void __launch_bounds__(256)
 absmax_mean_finish(const double* __restrict__ work, int64_t nchunks, int64_t nb, float* __restrict__ center)
 {
-    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    __shared__ double tile[kFinishTile];
     double total = 0.0;
-    for (int64_t c = 0; c < nchunks; c++) total = __dadd_rn(total, work[c]);
-    *center = __double2float_rn(__ddiv_rn(total, (double)nb));
+    for (int64_t c0 = 0; c0 < nchunks; c0 += kFinishTile) {
+        const int len = (int)(nchunks - c0 < kFinishTile ? nchunks - c0 : kFinishTile);
+        __syncthreads();
+        for (int i = threadIdx.x; i < len; i += blockDim.x) tile[i] = work[c0 + i];
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int i = 0; i < len; i++) total = __dadd_rn(total, tile[i]);
+    }
+    if (threadIdx.x == 0) *center = __double2float_rn(__ddiv_rn(total, (double)nb));
 }
 
 __global__ void __launch_bounds__(256)
@@ -134,7 +145,7 @@ bnbq_status launch_absmax_mean(const float* a, int64_t nb, double* work, float* 
     absmax_chunk_sums<<<(unsigned)nchunks, 256, 0, s>>>(a, nb, work);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "absmax_chunk_sums launch");
-    absmax_mean_finish<<<1, 32, 0, s>>>(work, nchunks, nb, center);
+    absmax_mean_finish<<<1, 256, 0, s>>>(work, nchunks, nb, center);
     return cuda_status(cudaGetLastError(), "absmax_mean_finish launch");
 }
 

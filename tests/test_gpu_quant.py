@@ -108,6 +108,25 @@ def test_other_codebooks(code_name):
     _check_full(code, x, 2048)
 
 
+@pytest.mark.parametrize("kind", ["crowded", "tiny"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_16_codes_outside_the_12_bit_table(kind, dtype):
+    """16-entry codebooks the 12-bit-prefix search cannot take: two midpoints in one of its
+    buckets (codes 0.5, 0.505, 0.51), or a midpoint below 2^-41 (the FMA quotient's safe range).
+    The kernel falls back to the 16-bit-prefix table or the midpoint walk; results as the
+    oracle's."""
+    base = np.concatenate([-np.linspace(1.0, 0.125, 7), [0.0]])
+    if kind == "crowded":
+        pos = [0.25, 0.5, 0.505, 0.51, 0.75, 0.875, 0.9375, 1.0]
+    else:
+        pos = [2.0 ** -45, 0.125, 0.25, 0.375, 0.5, 0.625, 0.75, 1.0]
+    code = torch.tensor(np.concatenate([base, pos]).astype(np.float32))
+    assert bq.bnbq_check_codebook(code) is None and code.numel() == 16
+    x = sweep_input(64 * 3000 + 19, dtype, f"16codes-{kind}")
+    for B in (64, 2048):
+        _check_full(code, x, B)
+
+
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 255, 256, 257, 2047, 2049, 4097, 8191])
 @pytest.mark.parametrize("code_name", ["signed", "nf4"])
 def test_small_and_ragged(n, code_name):
