@@ -23,7 +23,7 @@ OPTIMS = {"adamw": ADAMW, "adam": ADAM, "lion": LION, "momentum": MOMENTUM, "rms
 CODE_DYNAMIC_SIGNED, CODE_DYNAMIC_UNSIGNED, CODE_NF4, CODE_LINEAR, CODE_FP4 = 0, 1, 2, 3, 4
 CODE_KINDS = {"dynamic_signed": CODE_DYNAMIC_SIGNED, "dynamic_unsigned": CODE_DYNAMIC_UNSIGNED,
               "nf4": CODE_NF4, "linear": CODE_LINEAR, "fp4": CODE_FP4}
-FLAG_BAD_CODE, FLAG_NONFINITE = 0x1, 0x2
+FLAG_BAD_CODE, FLAG_NONFINITE, FLAG_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTED = ["bnbq_quantize_blockwise", "bnbq_dequantize_blockwise", "bnbq_step_8bit", "bnbq_step_8bit_noalloc",
             "bnbq_nested_workspace_bytes", "bnbq_quantize_absmax_nested", "bnbq_dequantize_absmax_nested",

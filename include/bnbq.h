@@ -23,7 +23,9 @@
  *  - No entry point aborts, throws, traps or waits on the device.  A codebook that fails the
  *    device-side check (strictly increasing, finite, within [-1, 1]) makes the kernel write
  *    nothing and sets BNBQ_FLAG_BAD_CODE; non-finite values met while building block scales set
- *    BNBQ_FLAG_NONFINITE.  Read the flags with bnbq_device_flags().
+ *    BNBQ_FLAG_NONFINITE.  Kernels wait only for their own bulk copies into shared memory, each
+ *    wait bounded (about a second); one that runs out sets BNBQ_FLAG_TIMEOUT.  Read the flags
+ *    with bnbq_device_flags().
  *  - Blocks have `blocksize` consecutive elements -- 64, 128, 256, 2048 or 4096 for quantize and
  *    dequantize, 256, 2048 or 4096 for the optimizer step; the last block of a tensor may be
  *    shorter; blocks never span two tensors.  Block b's scale is absmax[b].
@@ -77,6 +79,7 @@ typedef enum {
 /* device flag bits (bnbq_device_flags) */
 #define BNBQ_FLAG_BAD_CODE 0x1u  /* a codebook failed the device-side check; the kernel wrote nothing */
 #define BNBQ_FLAG_NONFINITE 0x2u /* a block scale (absmax) came out NaN or Inf */
+#define BNBQ_FLAG_TIMEOUT 0x4u   /* a kernel's bounded wait for its own copy ran out; its outputs are incomplete */
 
 /*
  * Block-wise quantization (abstract of "8-bit Optimizers via Block-wise Quantization";
