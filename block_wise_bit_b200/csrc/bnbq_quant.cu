@@ -19,6 +19,7 @@
 
 #include <mutex>
 
+#include "bnbq_async.cuh"
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 

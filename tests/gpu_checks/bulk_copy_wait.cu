@@ -1,4 +1,4 @@
-// Check of the library's bulk-copy helpers (bnbq_device.cuh): a 32 KB cp.async.bulk copy into
+// Check of the library's bulk-copy helpers (bnbq_async.cuh): a 32 KB cp.async.bulk copy into
 // shared memory completes its mbarrier and delivers the bytes, and a wait on a barrier phase that
 // never completes (a barrier that nothing arrives on) returns false after the wait budget instead
 // of spinning on, leaving the context usable for the next launch.
@@ -9,7 +9,7 @@
 #include <cstdio>
 #include <vector>
 
-#include "../../block_wise_bit_b200/csrc/bnbq_device.cuh"
+#include "../../block_wise_bit_b200/csrc/bnbq_async.cuh"
 
 namespace {
 

@@ -1,5 +1,5 @@
 """The bulk-copy helpers behind the staged quantize kernel (tests/gpu_checks/bulk_copy_wait.cu,
-built from the library's own device header): a 32 KB copy into shared memory completes its
+built from the library's own bulk-copy header): a 32 KB copy into shared memory completes its
 barrier with the right bytes, and a wait on a barrier that nothing arrives on gives up after its
 budget (about a second) and returns, the context staying usable."""
 import os
