@@ -134,8 +134,8 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
 template <int MODE>
 __device__ __forceinline__ uint32_t code_word(const CodeSmem& cs, float x)
 {
-    if constexpr (MODE == kSearchPrefix12)
-        return nearest_code_word12(cs.table, x);
+    if constexpr (MODE == kSearchPrefix11)
+        return nearest_code_word11(cs.table, x);
     else
         return nearest_code_word<MODE>(cs, x);
 }
@@ -433,11 +433,11 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
     }
     bool fast, general;
     if constexpr (K == 16) {
-        // 16 codes: the 12-bit-prefix table when no bucket of it holds two midpoints
+        // 16 codes: the 11-bit-prefix table when no bucket of it holds two midpoints
         if (!stage_one_code(cs, code, K, false, fast, general, flags)) return;
-        if (!__syncthreads_or(build_table12(cs.table, cs.mid, K))) {
+        if (!__syncthreads_or(build_table11(cs.table, cs.mid, K))) {
             __syncthreads();
-            quantize_run<B, BF16, WIDE, K, kSearchPrefix12, CENTER, STAGED>(cs, fast, A, n, absmax, out, red, flags,
+            quantize_run<B, BF16, WIDE, K, kSearchPrefix11, CENTER, STAGED>(cs, fast, A, n, absmax, out, red, flags,
                                                                             center, smem_raw);
             return;
         }

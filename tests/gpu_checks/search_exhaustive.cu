@@ -4,8 +4,8 @@
 //      q = #{ j : x > mid_j },  mid_j = fl32((code_j + code_{j+1}) / 2)  (sum formed in double),
 // with the midpoints formed on the host.  Each search mode is checked where it applies: the
 // one-load rule when no bucket holds two midpoints, the non-negative rule when every code is
-// >= 0, the midpoint walk always, and for a 16-entry codebook the 12-bit-prefix table
-// (build_table12 / nearest_code_word12) when none of its buckets holds two midpoints.
+// >= 0, the midpoint walk always, and for a 16-entry codebook the 11-bit-prefix table
+// (build_table11 / nearest_code_word11) when none of its buckets holds two midpoints.
 //
 // Usage: search_exhaustive <codebook file: K raw float32 values> <K>
 // Prints one line per mode and a final status line; exits 0 only if every checked mode matches.
@@ -20,26 +20,26 @@ namespace {
 
 constexpr uint32_t kHalfValues = 0x3F800000u + 1u;  // bit patterns 0 .. 0x3F800000 (+0 .. 1.0)
 
-__global__ void setup(const float* code, int K, float* mid, uint32_t* table, uint32_t* table12, int* flags)
+__global__ void setup(const float* code, int K, float* mid, uint32_t* table, uint32_t* table11, int* flags)
 {
     bool bad = false, tiny = false;
     bnbq::stage_midpoints(code, mid, K, bad, tiny);
     __syncthreads();
     const bool general = bnbq::build_bucket_entries(table + bnbq::kHalf, mid, K, -bnbq::kHalf, bnbq::kHalf - 1);
-    const bool general12 = K == 16 && bnbq::build_table12(table12, mid, K);
+    const bool general11 = K == 16 && bnbq::build_table11(table11, mid, K);
     const int g = __syncthreads_or(general);
-    const int g12 = __syncthreads_or(general12);
+    const int g11 = __syncthreads_or(general11);
     const int b = __syncthreads_or(bad);
     if (threadIdx.x == 0) {
         flags[0] = g;
         flags[1] = b;
-        flags[2] = g12;
+        flags[2] = g11;
     }
 }
 
 // One pass over every value: the reference count is formed once per value and compared with each
 // search mode that applies (check[m] != 0), mismatches counted per mode.
-__global__ void sweep(const uint32_t* table, const uint32_t* table12, const float* mid, const float* ref_mid, int K,
+__global__ void sweep(const uint32_t* table, const uint32_t* table11, const float* mid, const float* ref_mid, int K,
                       int4 check, unsigned long long* bad, unsigned* first)
 {
     __shared__ float rm[256];
@@ -57,7 +57,7 @@ __global__ void sweep(const uint32_t* table, const uint32_t* table12, const floa
         if (check.x) q[0] = bnbq::nearest_code_word<bnbq::kSearchSigned>(center, mid, x) >> 24;
         if (check.y) q[1] = bnbq::nearest_code_word<bnbq::kSearchNonNeg>(center, mid, x) >> 24;
         if (check.z) q[2] = bnbq::nearest_code_word<bnbq::kSearchGeneral>(center, mid, x) >> 24;
-        if (check.w) q[3] = bnbq::nearest_code_word12(table12, x) >> 24;
+        if (check.w) q[3] = bnbq::nearest_code_word11(table11, x) >> 24;
 #pragma unroll
         for (int m = 0; m < 4; m++)
             if (q[m] != r) {
@@ -91,20 +91,20 @@ int main(int argc, char** argv)
     }
 
     float *d_code = nullptr, *d_mid = nullptr, *d_ref = nullptr;
-    uint32_t *d_table = nullptr, *d_table12 = nullptr;
+    uint32_t *d_table = nullptr, *d_table11 = nullptr;
     int* d_flags = nullptr;
     unsigned long long* d_bad = nullptr;
     unsigned* d_first = nullptr;
     if (cudaMalloc(&d_code, 256 * sizeof(float)) != cudaSuccess || cudaMalloc(&d_mid, 256 * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&d_ref, 256 * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&d_table, bnbq::kTableSize * sizeof(uint32_t)) != cudaSuccess ||
-        cudaMalloc(&d_table12, bnbq::kTable12 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&d_table11, bnbq::kTable11 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&d_flags, 3 * sizeof(int)) != cudaSuccess || cudaMalloc(&d_bad, 4 * sizeof(*d_bad)) != cudaSuccess ||
         cudaMalloc(&d_first, 4 * sizeof(*d_first)) != cudaSuccess)
         return 3;
     cudaMemcpy(d_code, code.data(), K * sizeof(float), cudaMemcpyHostToDevice);
     cudaMemcpy(d_ref, ref_mid.data(), (K - 1) * sizeof(float), cudaMemcpyHostToDevice);
-    setup<<<1, 1024>>>(d_code, K, d_mid, d_table, d_table12, d_flags);
+    setup<<<1, 1024>>>(d_code, K, d_mid, d_table, d_table11, d_flags);
     cudaError_t e = cudaDeviceSynchronize();
     int flags[3] = {-1, -1, -1};
     std::vector<float> dev_mid(K);
@@ -112,23 +112,23 @@ int main(int argc, char** argv)
     cudaMemcpy(dev_mid.data(), d_mid, K * sizeof(float), cudaMemcpyDeviceToHost);
     bool mids_equal = true;
     for (int j = 0; j + 1 < K; j++) mids_equal = mids_equal && dev_mid[j] == ref_mid[j];
-    printf("setup status %s general %d bad %d nonneg %d prefix12-general %d midpoints %s\n", cudaGetErrorString(e),
+    printf("setup status %s general %d bad %d nonneg %d prefix11-general %d midpoints %s\n", cudaGetErrorString(e),
            flags[0], flags[1], nonneg ? 1 : 0, flags[2], mids_equal ? "equal" : "DIFFER");
     bool ok = e == cudaSuccess && flags[1] == 0 && mids_equal;
     if (ok) {
         // the one-load rule where no bucket holds two midpoints, the non-negative rule for a
         // codebook without negative codes, the midpoint walk always, and for 16 codes the
-        // 12-bit-prefix table where none of its buckets holds two midpoints
+        // 11-bit-prefix table where none of its buckets holds two midpoints
         const int4 check = make_int4(flags[0] == 0 ? 1 : 0, nonneg ? 1 : 0, 1, (K == 16 && flags[2] == 0) ? 1 : 0);
         cudaMemset(d_bad, 0, 4 * sizeof(*d_bad));
         cudaMemset(d_first, 0xff, 4 * sizeof(*d_first));
-        sweep<<<148 * 8, 256>>>(d_table, d_table12, d_mid, d_ref, K, check, d_bad, d_first);
+        sweep<<<148 * 8, 256>>>(d_table, d_table11, d_mid, d_ref, K, check, d_bad, d_first);
         e = cudaDeviceSynchronize();
         unsigned long long bad[4] = {~0ull, ~0ull, ~0ull, ~0ull};
         unsigned first[4] = {0, 0, 0, 0};
         cudaMemcpy(bad, d_bad, sizeof(bad), cudaMemcpyDeviceToHost);
         cudaMemcpy(first, d_first, sizeof(first), cudaMemcpyDeviceToHost);
-        const char* names[4] = {"signed", "nonneg", "general", "prefix12"};
+        const char* names[4] = {"signed", "nonneg", "general", "prefix11"};
         const int on[4] = {check.x, check.y, check.z, check.w};
         for (int m = 0; m < 4; m++)
             if (on[m]) {

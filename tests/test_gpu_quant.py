@@ -124,16 +124,19 @@ def test_other_codebooks(code_name):
     _check_full(code, x, 2048)
 
 
-@pytest.mark.parametrize("kind", ["crowded", "tiny"])
+@pytest.mark.parametrize("kind", ["crowded", "crowded11", "tiny"])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_16_codes_outside_the_12_bit_table(kind, dtype):
-    """16-entry codebooks the 12-bit-prefix search cannot take: two midpoints in one of its
-    buckets (codes 0.5, 0.505, 0.51), or a midpoint below 2^-41 (the FMA quotient's safe range).
-    The kernel falls back to the 16-bit-prefix table or the midpoint walk; results as the
-    oracle's."""
+def test_16_codes_outside_the_prefix_table(kind, dtype):
+    """16-entry codebooks the 11-bit-prefix search cannot take: two midpoints in one of its
+    buckets (codes 0.5, 0.505, 0.51, which a 12-bit prefix would not separate either, or 0.5,
+    0.53, 0.6, which it would), where the kernel falls back to the 16-bit-prefix table or the
+    midpoint walk; and a midpoint below 2^-41 (outside the FMA quotient's safe range), where it
+    divides with IEEE division.  Results as the oracle's."""
     base = np.concatenate([-np.linspace(1.0, 0.125, 7), [0.0]])
     if kind == "crowded":
         pos = [0.25, 0.5, 0.505, 0.51, 0.75, 0.875, 0.9375, 1.0]
+    elif kind == "crowded11":
+        pos = [0.25, 0.5, 0.53, 0.6, 0.75, 0.875, 0.9375, 1.0]
     else:
         pos = [2.0 ** -45, 0.125, 0.25, 0.375, 0.5, 0.625, 0.75, 1.0]
     code = torch.tensor(np.concatenate([base, pos]).astype(np.float32))

@@ -36,4 +36,4 @@ def test_search_exhaustive(checker, tmp_path, kind):
     assert out.returncode == 0 and "result ok" in out.stdout, out.stdout + out.stderr
     assert "midpoints equal" in out.stdout and "mode general status no error mismatches 0" in out.stdout
     if code.size == 16:  # the quantize kernel's search for 16 codes
-        assert "mode prefix12 status no error mismatches 0" in out.stdout, out.stdout
+        assert "mode prefix11 status no error mismatches 0" in out.stdout, out.stdout
