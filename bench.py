@@ -177,6 +177,39 @@ def bench_quant(args, base):
         print(json.dumps(out), flush=True)
 
 
+def bench_hbm_mix(args, base):
+    """Context for the rooflines of write-heavy kernels (--workload hbm_mix): the HBM rate that
+    torch's own kernels reach on 512 MiB buffers for a write-only stream (fill) and a 50/50
+    read-write stream (copy), CUDA events, median over the timed calls.  None of this library's
+    kernels run."""
+    import torch
+    dev = torch.device("cuda", 0)
+    n = 1 << 28
+    a = torch.empty(n, dtype=torch.bfloat16, device=dev).normal_()
+    b = torch.empty_like(a)
+    stream = torch.cuda.current_stream(dev)
+    peak, kind = measured_peaks()
+    res = {}
+    for name, fn, nbytes in (("write_only_fill", lambda: b.fill_(1.5), 2 * n), ("copy", lambda: b.copy_(a), 4 * n)):
+        for _ in range(args.warmup):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+        res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 4),
+                     "bytes": nbytes}
+    out = dict(base, metric="HBM rate of torch fill / copy (context)", unit="GB/s", value=res["write_only_fill"]["GB/s"],
+               n_gpus=1, steps=args.steps, warmup=args.warmup, ms_per_step=res["write_only_fill"]["ms"], dtype="bf16",
+               config={"workload": "hbm_mix", "bytes_per_buffer": 2 * n}, peak_gbs=peak, peak_source=kind,
+               gpu_launches=0, **res)
+    print(json.dumps(out), flush=True)
+
+
 def bench_zero1(args, base, shape, optim, seed, hp, outlier):
     """ZeRO-1 data-parallel step over the whole list on ``world`` ranks: every rank holds the full
     flat parameters and its own full bf16 gradient; per step the gradients are reduce-scattered in
@@ -500,7 +533,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS) + ["quant_sweep"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS) + ["quant_sweep", "hbm_mix"],
                     default="llama7b_adamw")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
@@ -520,7 +553,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.workload.startswith("quant"):
+    if args.workload.startswith("quant") or args.workload == "hbm_mix":
         shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS["llama7b_adamw"]
     else:
         shape, optim, seed, hp, (ofrac, oscale) = WORKLOADS[args.workload]
@@ -565,6 +598,8 @@ def main():
 
     if args.workload.startswith("quant"):
         return bench_quant(args, base)
+    if args.workload == "hbm_mix":
+        return bench_hbm_mix(args, base)
     if args.zero1:
         return bench_zero1(args, base, shape, optim, seed, hp, (ofrac, oscale))
 
