@@ -95,7 +95,9 @@ typedef enum {
  * Element i of block b gets q = #{ j : A_i/absmax[b] > mid_j } with
  * mid_j = fl32((code_j + code_{j+1})/2): the nearest code, a tie going to the lower code; a
  * block whose absmax is 0 maps to the code nearest 0.  The division is correctly rounded.
- * n == 0 is a no-op.
+ * n == 0 is a no-op.  The environment variable BNBQ_QUANT_MAX_CTAS=<k>, read at each call, caps
+ * the kernel's grid at k CTAs (a testing aid: every CTA then takes many tiles; unset = one or two
+ * CTAs per SM).
  */
 BNBQ_API bnbq_status bnbq_quantize_blockwise(const float* code, int code_size, const void* A,
                                     bnbq_dtype a_dtype, int64_t n, int blocksize, float* absmax,
