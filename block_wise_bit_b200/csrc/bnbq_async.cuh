@@ -52,6 +52,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return done != 0;
 }
 
+// Hint: bring `bytes` (a multiple of 16; address 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void l2_prefetch(const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Wait for the phase of parity `parity` to complete; false if it has not within kWaitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
 {

@@ -43,8 +43,9 @@ struct QGeom {
     static constexpr int kGroupWarps = G >= 32 ? G / 32 : 1;
     static constexpr size_t kSmem = sizeof(CodeSmem) + sizeof(float) * kGroups * 2 * kGroupWarps;
     static_assert(G >= 1 && kQThreads % G == 0 && (!WIDE || BF16), "group geometry");
-    // Staged variant (fp32 input): a CTA's blocks of one pass form a tile of kGroups * B
-    // elements (32 KB), copied into shared memory one or two tiles ahead of the threads.
+    // A CTA's blocks of one pass form a tile of kGroups * B elements (32 KB of input for either
+    // dtype).  Staged variant (fp32 input): tiles are copied into shared memory one or two tiles
+    // ahead of the threads; aligned bf16 input: the next tile is prefetched into L2.
     static constexpr int kES = BF16 ? 2 : 4;
     static constexpr int64_t kTileElems = (int64_t)kGroups * B;
     static constexpr uint32_t kTileBytes = (uint32_t)(kTileElems * kES);
@@ -168,16 +169,25 @@ __device__ __forceinline__ uint32_t codes4(const CodeSmem& cs, const BlockScale&
     return pack_top_bytes(w[0], w[1], w[2], w[3]);
 }
 
+// Four codes below 16, one per byte (c0 | c1 << 8 | c2 << 16 | c3 << 24), merged into nibble
+// pairs: times 4097 adds a copy shifted left by 12 bits (no two nibbles overlap, so nothing
+// carries), which puts c0 << 4 | c1 in byte 1 and c2 << 4 | c3 in byte 3.
+__device__ __forceinline__ uint32_t nibble_pairs(uint32_t bytes4) { return bytes4 * 4097u; }
+
 // The 4-bit codes of 4 consecutive elements packed two per byte (even element in the high nibble)
-// in the low 16 bits, formed with integer multiply-adds (codes below 16).
+// in the low 16 bits.
 template <int MODE, bool FAST>
 __device__ __forceinline__ uint32_t nibbles4(const CodeSmem& cs, const BlockScale& sc, const float* x)
 {
-    uint32_t w[4];
-    words4<MODE, FAST>(cs, sc, x, w);
-    const uint32_t b0 = (w[0] >> 24) * 16u + (w[1] >> 24);
-    const uint32_t b1 = (w[2] >> 24) * 16u + (w[3] >> 24);
-    return b1 * 256u + b0;
+    return __byte_perm(nibble_pairs(codes4<MODE, FAST>(cs, sc, x)), 0u, 0x0031u);
+}
+
+// The same for 8 consecutive elements: four packed bytes.
+template <int MODE, bool FAST>
+__device__ __forceinline__ uint32_t nibbles8(const CodeSmem& cs, const BlockScale& sc, const float* x)
+{
+    return __byte_perm(nibble_pairs(codes4<MODE, FAST>(cs, sc, x)), nibble_pairs(codes4<MODE, FAST>(cs, sc, x + 4)),
+                       0x7531u);
 }
 
 // Normalise, search and store one block's chunks (FAST: FMA quotient, else IEEE division; FULL:
@@ -196,8 +206,7 @@ __device__ __forceinline__ void quantize_store(const CodeSmem& cs, const BlockSc
         if constexpr (K == 16) {
             if (FULL || e + CW <= n) {
                 if constexpr (CW == 8)
-                    st_stream_u32(out + (e >> 1), nibbles4<MODE, FAST>(cs, sc, &v[j][4]) * 65536u +
-                                                      nibbles4<MODE, FAST>(cs, sc, &v[j][0]));
+                    st_stream_u32(out + (e >> 1), nibbles8<MODE, FAST>(cs, sc, &v[j][0]));
                 else
                     *reinterpret_cast<uint16_t*>(out + (e >> 1)) = (uint16_t)nibbles4<MODE, FAST>(cs, sc, &v[j][0]);
                 continue;
@@ -309,7 +318,14 @@ __device__ __forceinline__ void quantize_loop(const CodeSmem& cs, bool fast, con
     const float off = CENTER ? __ldg(center) : 0.0f;
     int parity = 0;
 
+    int64_t tile = blockIdx.x;  // the CTA's blocks of this pass: tile kGroups * tile .. + kGroups - 1
     for (int64_t b = (int64_t)blockIdx.x * Geo::kGroups + gi; b < nb; b += (int64_t)gridDim.x * Geo::kGroups) {
+        if constexpr (BF16 && WIDE) {  // 16-byte aligned bf16: the CTA's next tile into L2 (a hint)
+            const int64_t next = tile + gridDim.x;
+            if (threadIdx.x == 0 && (next + 1) * Geo::kTileElems <= n)
+                l2_prefetch(static_cast<const char*>(A) + next * (int64_t)Geo::kTileBytes, Geo::kTileBytes);
+            tile = next;
+        }
         if ((b + 1) * B <= n)  // group-uniform: every thread of the group holds the same block
             quantize_block<B, BF16, WIDE, K, MODE, CENTER, true>(cs, fast, A, n, absmax, out, red, flags, off, b, gi,
                                                                  tg, lane, gmask, parity);
@@ -689,7 +705,9 @@ bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax,
 }
 
 // bf16 input 16-byte aligned, with codes aligned for 8 (8-bit) or 4 (4-bit) bytes per store:
-// 8-element chunks; otherwise 4-element chunks.
+// 8-element chunks, and thread 0 of each CTA prefetches the CTA's next 32 KB tile into L2 at the
+// start of each pass (measured on B200 at 2^28 elements: 8-bit codes 4-7% faster, NF4 unchanged;
+// two tiles ahead was slower for 8-bit codes); otherwise 4-element chunks.
 template <int B, bool BF16>
 bnbq_status launch_q_k(const float* code, int K, const void* A, int64_t n, float* absmax,
                        uint8_t* out, cudaStream_t s)
