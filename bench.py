@@ -671,7 +671,10 @@ def main():
                 "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload, alg),
                 "peak_source": f"{peak_kind} HBM copy bandwidth", "algorithmic_bytes_per_launch": alg,
                 "kernel": f"step_kernel<{optim}, 2048>", "avg_launch_ms": round(avg_launch_ms, 4),
+                "median_launch_ms": round(statistics.median(launch_ms), 4),
                 "min_launch_ms": round(min(launch_ms), 4), "max_launch_ms": round(max(launch_ms), 4)}
+    if roofline["traffic"] is not None:  # the same rate from the ncu DRAM bytes of a captured launch
+        roofline["dram_gbs"] = round(roofline["traffic"] / (avg_launch_ms / 1e3) / 1e9, 1)
     if args.series:
         roofline["launch_ms"] = [round(x, 3) for x in launch_ms]
         k = max(1, len(launch_ms) // 3)
