@@ -169,7 +169,8 @@ def test_small_and_ragged_bf16(n, code_name):
 @pytest.mark.parametrize("code_name", ["signed", "nf4"])
 def test_bf16_input_and_codes_at_narrow_alignment(code_name):
     """bf16 input only 8-byte aligned and codes only as aligned as the interface asks (4 bytes for
-    8-bit codes, 2 for 4-bit): the kernel falls back to 4-element chunks; results as the oracle's."""
+    8-bit codes, 2 for 4-bit): quantize falls back to 4-element chunks and dequantize to 16-bit
+    code loads; results as the oracle's."""
     code = _codes()[code_name]
     n, B = 64 * 1000 + 37, 64
     K = code.numel()
@@ -187,6 +188,12 @@ def test_bf16_input_and_codes_at_narrow_alignment(code_name):
     a_or, q_or = oracle.quantize_blockwise(code.numpy(), parity.to_np(x), B)
     np.testing.assert_array_equal(parity.to_np(a).view(np.uint32), a_or.view(np.uint32))
     np.testing.assert_array_equal(parity.to_np(q), q_or)
+    for dt in (torch.float32, torch.bfloat16):
+        y = bq.bnbq_dequantize_blockwise(code.to(DEV), q, a, n, B, out_dtype=dt)
+        y_or = oracle.dequantize_blockwise(code.numpy(), q_or, a_or, n, B, out_bf16=(dt == torch.bfloat16))
+        gy = parity.to_np(y)
+        np.testing.assert_array_equal(gy.view(np.uint32) if dt == torch.float32 else gy,
+                                      y_or.view(np.uint32) if dt == torch.float32 else y_or)
 
 
 def test_empty_is_noop():
