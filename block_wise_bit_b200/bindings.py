@@ -327,6 +327,9 @@ def bnbq_step_8bit_noalloc(opt: str | int, tensors: Sequence[TensorState] | ctyp
 
 
 def bnbq_device_flags(clear: bool = False) -> int:
+    """The calling device's flag word (synchronizes the device): FLAG_BAD_CODE (a codebook failed
+    the device-side check), FLAG_NONFINITE (a block scale came out NaN or Inf), FLAG_TIMEOUT (a
+    kernel's bounded wait for its own bulk copy ran out); ``clear`` resets it."""
     v = ctypes.c_uint32(0)
     _check(lib().bnbq_device_flags(ctypes.byref(v), int(clear)))
     return int(v.value)

@@ -37,6 +37,18 @@ def test_library_exports_every_declared_symbol():
     assert B.bnbq_version() == "0.1.0"
 
 
+def test_flag_bits_match_the_header():
+    """The binding's flag constants and the device code's flag bits are the header's."""
+    src = open(HEADER).read()
+    defs = {m.group(1): int(m.group(2), 16) for m in re.finditer(r"#define BNBQ_FLAG_([A-Z_]+) (0x[0-9a-fA-F]+)u", src)}
+    assert defs == {"BAD_CODE": B.FLAG_BAD_CODE, "NONFINITE": B.FLAG_NONFINITE, "TIMEOUT": B.FLAG_TIMEOUT}
+    dev = ""
+    for f in ("bnbq_device.cuh", "bnbq_async.cuh"):
+        dev += open(os.path.join(ROOT, "block_wise_bit_b200", "csrc", f)).read()
+    kdefs = {m.group(1): int(m.group(2), 16) for m in re.finditer(r"constexpr unsigned kFlag(\w+) = (0x[0-9a-fA-F]+)u", dev)}
+    assert kdefs == {"BadCode": defs["BAD_CODE"], "NonFinite": defs["NONFINITE"], "Timeout": defs["TIMEOUT"]}
+
+
 def test_only_bnbq_symbols_exported():
     out = os.popen(f"nm -D --defined-only {B.library_path()}").read().split("\n")
     funcs = [ln.split()[-1] for ln in out if " T " in ln]
