@@ -11,107 +11,126 @@
 // The mean is a plain double sum in a fixed order -- chunks of kNestChunk consecutive scales,
 // each summed in index order, then the chunk sums in index order -- divided by nb in double and
 // rounded once to binary32, so every run (and the CPU restatement) gets the same offset.  A
-// chunk whose index-order sum is exact (see absmax_chunk_sums) is added up in parallel.
+// chunk whose index-order sum is exact is added up in parallel, and so are the chunk sums when the
+// whole array's sum is exact (absmax_mean_kernel).
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
 
 namespace bnbq {
 namespace {
 
-// min / max of an int over the CTA (every thread calls; every thread gets the result)
-__device__ __forceinline__ int min_over_block(int v)
-{
-    __shared__ int r[32];
-    for (int off = 16; off > 0; off >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, off));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) r[threadIdx.x >> 5] = v;
-    __syncthreads();
-    v = r[0];
-    for (int w = 1; w < (int)(blockDim.x >> 5); w++) v = min(v, r[w]);
-    return v;
-}
-
-__device__ __forceinline__ int max_over_block(int v)
-{
-    return -min_over_block(-v);
-}
-
-// One CTA per chunk: the chunk is staged in shared memory with coalesced loads and summed in
-// double.  The definition is the index-order sum, s = ((a0 + a1) + a2) + ...; when every partial
-// sum of that order is exact the result does not depend on the order, and the CTA adds in
-// parallel.  That holds when the ulps of the chunk's non-zero values span at most 2^17: every
-// value is then an integer multiple of the smallest ulp U and below 2^24 times the largest, so
-// the sum of at most 4096 = 2^12 of them stays below 2^(24+12+17) U = 2^53 U, an integer number
-// of U's that a double holds exactly.  Otherwise (a wider spread, or a NaN or infinity) one thread
-// adds in index order.
-constexpr int kSumThreads = 256;
+// The mean in one launch.  One CTA per chunk of kNestChunk scales; each thread takes every
+// kMeanThreads-th value of the chunk (coalesced loads, kept in registers) and forms, in one pass,
+// the range of the values' ulp exponents and their double sum.  The definition is the index-order
+// sum, s = ((a0 + a1) + a2) + ...; when every partial sum of that order is exact the result does
+// not depend on the order, and the CTA adds in parallel.  That holds when the ulps of the chunk's
+// non-zero values span at most 2^17: every value is then an integer multiple of the smallest ulp U
+// and below 2^24 times the largest, so the sum of at most 4096 = 2^12 of them stays below
+// 2^(24+12+17) U = 2^53 U, an integer number of U's that a double holds exactly.  Otherwise (a
+// wider spread, or a NaN or infinity) one thread adds the chunk in index order.
+// Each CTA stores its chunk sum and exponent range, and the last CTA to finish (a counter in the
+// workspace, zeroed before the launch) adds the chunk sums: in parallel when the sum over the
+// whole array is exact by the same argument -- nb values whose ulps span at most 2^d, with
+// nb * 2^(24+d) <= 2^53 -- else in index order by one thread.  No CTA waits for another.
+constexpr int kMeanThreads = 256;
+constexpr int kMeanWarps = kMeanThreads / 32;
+constexpr int kPerThread = kNestChunk / kMeanThreads;
+constexpr int kNoValue = 255;      // exponent-range sentinel: no non-zero value
+constexpr int kNotFinite = 1000;   // exponent of a NaN or infinity: forces the ordered sums
 
 __device__ __forceinline__ int ulp_exponent(float x)  // biased exponent of x's ulp; 1 for subnormals
 {
     const int e = (int)((__float_as_uint(x) >> 23) & 0xffu);
-    return e == 0 ? 1 : e;
+    return e == 0 ? 1 : (e == 0xff ? kNotFinite : e);
 }
 
-__global__ void __launch_bounds__(kSumThreads)
-absmax_chunk_sums(const float* __restrict__ a, int64_t nb, double* __restrict__ work)
+// CTA-wide min of lo, max of hi and sum of s; every thread gets the results.
+__device__ __forceinline__ void cta_reduce(int& lo, int& hi, double& s)
 {
-    __shared__ float chunk[kNestChunk];
-    __shared__ double part[kSumThreads / 32];
+    __shared__ int rlo[kMeanWarps], rhi[kMeanWarps];
+    __shared__ double rs[kMeanWarps];
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    __syncthreads();  // the arrays may still be read from a previous call
+    if ((threadIdx.x & 31) == 0) {
+        rlo[threadIdx.x >> 5] = lo;
+        rhi[threadIdx.x >> 5] = hi;
+        rs[threadIdx.x >> 5] = s;
+    }
+    __syncthreads();
+    lo = rlo[0];
+    hi = rhi[0];
+    s = rs[0];
+    for (int w = 1; w < kMeanWarps; w++) {
+        lo = min(lo, rlo[w]);
+        hi = max(hi, rhi[w]);
+        s = __dadd_rn(s, rs[w]);
+    }
+}
+
+__device__ __forceinline__ bool sum_is_exact(int lo, int hi, int log2_count)
+{
+    return lo == kNoValue || (hi < kNotFinite && hi - lo + 24 + log2_count <= 53);
+}
+
+__global__ void __launch_bounds__(kMeanThreads)
+absmax_mean_kernel(const float* __restrict__ a, int64_t nb, double* __restrict__ sums, int2* __restrict__ range,
+                   unsigned* __restrict__ counter, float* __restrict__ center)
+{
+    __shared__ bool last;
     const int64_t start = (int64_t)blockIdx.x * kNestChunk;
     const int len = (int)((nb - start < kNestChunk) ? nb - start : kNestChunk);
-    for (int i = threadIdx.x; i < len; i += blockDim.x) chunk[i] = __ldg(a + start + i);
-    __syncthreads();
-    // ulp exponent range of the non-zero values (a NaN or infinity forces the ordered sum)
-    // (threads take every kSumThreads-th value: consecutive threads read consecutive words, so the
-    // shared-memory reads never conflict; the exact sum below does not depend on the order)
-    int emin = 255, emax = 0;
-    for (int i = threadIdx.x; i < len; i += kSumThreads) {
-        const float x = chunk[i];
-        if (x == 0.0f) continue;
-        const int e = ulp_exponent(x);
-        emin = min(emin, e);
-        emax = max(emax, (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u ? 1000 : e);
-    }
-    emin = __syncthreads_and(emin == 255) ? 0 : min_over_block(emin);
-    emax = max_over_block(emax);
-    const bool exact = emax - emin <= 17;
-    if (exact) {  // every order gives the same (exact) sum
-        double s = 0.0;
-        for (int i = threadIdx.x; i < len; i += kSumThreads) s = __dadd_rn(s, (double)chunk[i]);
-        for (int off = 16; off > 0; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
-        if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double t = 0.0;
-            for (int w = 0; w < kSumThreads / 32; w++) t = __dadd_rn(t, part[w]);
-            work[blockIdx.x] = t;
-        }
-        return;
-    }
-    if (threadIdx.x != 0) return;
+    int lo = kNoValue, hi = 0;
     double s = 0.0;
-    for (int i = 0; i < len; i++) s = __dadd_rn(s, (double)chunk[i]);
-    work[blockIdx.x] = s;
-}
-
-// The chunk sums in index order: the CTA stages them in shared memory with coalesced loads, a
-// tile at a time, and one thread adds them up (the order is part of the definition).
-constexpr int kFinishTile = 2048;
-
-__global__ void __launch_bounds__(256)
-absmax_mean_finish(const double* __restrict__ work, int64_t nchunks, int64_t nb, float* __restrict__ center)
-{
-    __shared__ double tile[kFinishTile];
-    double total = 0.0;
-    for (int64_t c0 = 0; c0 < nchunks; c0 += kFinishTile) {
-        const int len = (int)(nchunks - c0 < kFinishTile ? nchunks - c0 : kFinishTile);
-        __syncthreads();
-        for (int i = threadIdx.x; i < len; i += blockDim.x) tile[i] = work[c0 + i];
-        __syncthreads();
-        if (threadIdx.x == 0)
-            for (int i = 0; i < len; i++) total = __dadd_rn(total, tile[i]);
+#pragma unroll
+    for (int k = 0; k < kPerThread; k++) {
+        const int i = (int)threadIdx.x + k * kMeanThreads;
+        if (i < len) {
+            const float x = __ldg(a + start + i);
+            if (x != 0.0f) {
+                const int e = ulp_exponent(x);
+                lo = min(lo, e);
+                hi = max(hi, e);
+            }
+            s = __dadd_rn(s, (double)x);
+        }
     }
-    if (threadIdx.x == 0) *center = __double2float_rn(__ddiv_rn(total, (double)nb));
+    cta_reduce(lo, hi, s);
+    if (threadIdx.x == 0) {
+        if (!sum_is_exact(lo, hi, 12)) {  // the chunk in index order
+            s = 0.0;
+            for (int i = 0; i < len; i++) s = __dadd_rn(s, (double)__ldg(a + start + i));
+        }
+        sums[blockIdx.x] = s;
+        range[blockIdx.x] = make_int2(lo, hi);
+        __threadfence();
+        last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!last) return;
+    // the last CTA: every other CTA's chunk sum and range are written (fence before the count)
+    __threadfence();
+    const int nchunks = (int)gridDim.x;
+    lo = kNoValue;
+    hi = 0;
+    s = 0.0;
+    for (int c = threadIdx.x; c < nchunks; c += kMeanThreads) {
+        const int2 r = __ldcg(range + c);
+        lo = min(lo, r.x);
+        hi = max(hi, r.y);
+        s = __dadd_rn(s, __ldcg(sums + c));
+    }
+    cta_reduce(lo, hi, s);
+    if (threadIdx.x == 0) {
+        int log2_nb = 0;
+        while ((1ll << log2_nb) < nb) log2_nb++;
+        if (!sum_is_exact(lo, hi, log2_nb)) {  // the chunk sums in index order
+            s = 0.0;
+            for (int c = 0; c < nchunks; c++) s = __dadd_rn(s, __ldcg(sums + c));
+        }
+        *center = __double2float_rn(__ddiv_rn(s, (double)nb));
+    }
 }
 
 __global__ void __launch_bounds__(256)
@@ -141,12 +160,14 @@ bool aligned_n(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>
 
 bnbq_status launch_absmax_mean(const float* a, int64_t nb, double* work, float* center, cudaStream_t s)
 {
+    // work: nchunks chunk sums (double), nchunks exponent ranges (int2), the finish counter
     const int64_t nchunks = (nb + kNestChunk - 1) / kNestChunk;
-    absmax_chunk_sums<<<(unsigned)nchunks, 256, 0, s>>>(a, nb, work);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_status(e, "absmax_chunk_sums launch");
-    absmax_mean_finish<<<1, 256, 0, s>>>(work, nchunks, nb, center);
-    return cuda_status(cudaGetLastError(), "absmax_mean_finish launch");
+    int2* range = reinterpret_cast<int2*>(work + nchunks);
+    unsigned* counter = reinterpret_cast<unsigned*>(range + nchunks);
+    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_status(e, "mean counter reset");
+    absmax_mean_kernel<<<(unsigned)nchunks, kMeanThreads, 0, s>>>(a, nb, work, range, counter, center);
+    return cuda_status(cudaGetLastError(), "absmax_mean_kernel launch");
 }
 
 bnbq_status launch_unnest(const uint8_t* qabs, const float* absmax2, const float* center, const float* code2,
@@ -163,7 +184,8 @@ using namespace bnbq;
 extern "C" BNBQ_API int64_t bnbq_nested_workspace_bytes(int64_t nb)
 {
     if (nb <= 0) return 0;
-    return (int64_t)sizeof(double) * ((nb + kNestChunk - 1) / kNestChunk);
+    const int64_t nchunks = (nb + kNestChunk - 1) / kNestChunk;
+    return (int64_t)(sizeof(double) + sizeof(int2)) * nchunks + 8;  // sums, exponent ranges, counter
 }
 
 extern "C" BNBQ_API bnbq_status bnbq_quantize_absmax_nested(const float* absmax, int64_t nb, const float* code2,

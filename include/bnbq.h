@@ -126,7 +126,7 @@ BNBQ_API bnbq_status bnbq_dequantize_blockwise(const float* code, int code_size,
  *   code2     device, 256 fp32 (the signed dynamic code is the intended one)
  *   workspace device, bnbq_nested_workspace_bytes(nb) bytes, 8-byte aligned, caller-owned;
  *             its contents are scratch.  absmax must be 16-byte aligned.
- * Asynchronous on `stream`; three kernel launches.
+ * Asynchronous on `stream`; a 4-byte memset of the workspace and two kernel launches.
  */
 BNBQ_API int64_t bnbq_nested_workspace_bytes(int64_t nb);
 BNBQ_API bnbq_status bnbq_quantize_absmax_nested(const float* absmax, int64_t nb, const float* code2,

@@ -107,8 +107,8 @@ def test_nested_argument_checks():
     """Nested quantization of block scales: checks before any CUDA call."""
     L = B.lib()
     assert L.bnbq_nested_workspace_bytes(0) == 0
-    assert L.bnbq_nested_workspace_bytes(1) == 8
-    assert L.bnbq_nested_workspace_bytes(4096) == 8 and L.bnbq_nested_workspace_bytes(4097) == 16
+    assert L.bnbq_nested_workspace_bytes(1) == 24          # chunk sum, exponent range, counter
+    assert L.bnbq_nested_workspace_bytes(4096) == 24 and L.bnbq_nested_workspace_bytes(4097) == 40
     q = L.bnbq_quantize_absmax_nested
     assert q(0x1000, -1, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == B.EINVAL
     assert q(0x1000, 10, None, 0x3000, 0x4000, 0x5000, 0x6000, None) == B.EINVAL        # no code2

@@ -66,6 +66,21 @@ def test_nest_absmax_mean_any_spread(nb):
     np.testing.assert_array_equal(parity.to_np(a2).view(np.uint32), a2_or.view(np.uint32))
 
 
+@pytest.mark.parametrize("nb", [8192 + 5, 70001, 1 << 20])
+def test_nest_absmax_mean_narrow_scales(nb):
+    """Scales within a factor 8 of each other (ulps spanning at most 2^3): the sum over the whole
+    array is exact, so the last CTA adds the chunk sums in parallel; with zeros mixed in.  The
+    offset must equal the oracle's index-order sum."""
+    code2 = bq.bnbq_codebook("dynamic_signed")
+    a = W.log_uniform(nb, 0.5, 4.0, DEV, "nested-narrow", nb)
+    a[::61] = 0.0
+    qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2.to(DEV), a)
+    q_or, a2_or, off_or = oracle.nest_absmax(parity.to_np(a), code2.numpy())
+    assert parity.to_np(off).view(np.uint32)[0] == np.float32(off_or).view(np.uint32)
+    np.testing.assert_array_equal(parity.to_np(qabs), q_or)
+    np.testing.assert_array_equal(parity.to_np(a2).view(np.uint32), a2_or.view(np.uint32))
+
+
 def test_nest_empty_and_equal_scales():
     code2 = bq.bnbq_codebook("dynamic_signed").to(DEV)
     qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2, torch.empty(0, device=DEV))
