@@ -676,6 +676,17 @@ int quant_cta_cap()
     return (end && *end == 0 && c > 0 && c < (1l << 30)) ? (int)c : 0;
 }
 
+// The size from which aligned fp32 input is staged: BNBQ_QUANT_STAGE_FROM=<elements> (read at
+// each launch; a testing aid, e.g. 0 to stage every size) or the measured default.
+int64_t quant_stage_from(int64_t dflt)
+{
+    const char* v = getenv("BNBQ_QUANT_STAGE_FROM");
+    if (!v || !*v) return dflt;
+    char* end = nullptr;
+    const long long c = strtoll(v, &end, 10);
+    return (end && *end == 0 && c >= 0) ? (int64_t)c : dflt;
+}
+
 template <int B, bool BF16, bool WIDE, int K, bool CENTER, bool STAGED>
 bnbq_status launch_q_s(const float* code, const void* A, int64_t n, float* absmax, uint8_t* out,
                        cudaStream_t s, const float* center)
@@ -711,18 +722,20 @@ bnbq_status launch_q_s(const float* code, const void* A, int64_t n, float* absma
     return cuda_status(cudaGetLastError(), "quantize_kernel launch");
 }
 
-// fp32 input 16-byte aligned and at least one whole tile: the staged kernel; otherwise plain
-// loads.  Measured on B200 (2^28 elements): staging gains 2-5% for fp32 input; for bf16 input it
-// lost 2-4%, because the kernel is bound by the shared-memory data pipe (the table lookups'
-// bank conflicts) and the ALU rather than by load latency, and reading the stage from shared
-// memory adds about 15% to that pipe's wavefronts.
+// Large aligned fp32 input: the staged kernel; otherwise plain loads.  Measured on B200 (blocksize
+// 2048): with 8-bit codes staging is 1-3% faster from 2^26 elements on and up to 6% slower below
+// (its first tiles wait for their copies); with 4-bit codes it is 2-3% faster at 2^28 but 5-7%
+// slower at 2^27, hence the thresholds.  For bf16 input it lost 2-4% at every size: that kernel
+// is bound by the shared-memory data pipe (the table lookups' bank conflicts) and the ALU rather
+// than by load latency, and reading the stage back adds about 15% to the data pipe's wavefronts.
 template <int B, bool BF16, bool WIDE, int K, bool CENTER = false>
 bnbq_status launch_q(const float* code, const void* A, int64_t n, float* absmax, uint8_t* out,
                      cudaStream_t s, const float* center = nullptr)
 {
-    using Geo = QGeom<B, BF16, WIDE>;
     if constexpr (!BF16) {
-        if ((reinterpret_cast<uintptr_t>(A) & 15u) == 0 && n >= Geo::kTileElems)
+        using Geo = QGeom<B, BF16, WIDE>;
+        const int64_t from = quant_stage_from(K == 256 ? (1ll << 26) : (1ll << 28));
+        if ((reinterpret_cast<uintptr_t>(A) & 15u) == 0 && n >= from && n >= Geo::kTileElems)
             return launch_q_s<B, BF16, WIDE, K, CENTER, true>(code, A, n, absmax, out, s, center);
     }
     return launch_q_s<B, BF16, WIDE, K, CENTER, false>(code, A, n, absmax, out, s, center);

@@ -95,9 +95,10 @@ typedef enum {
  * Element i of block b gets q = #{ j : A_i/absmax[b] > mid_j } with
  * mid_j = fl32((code_j + code_{j+1})/2): the nearest code, a tie going to the lower code; a
  * block whose absmax is 0 maps to the code nearest 0.  The division is correctly rounded.
- * n == 0 is a no-op.  The environment variable BNBQ_QUANT_MAX_CTAS=<k>, read at each call, caps
- * the kernel's grid at k CTAs (a testing aid: every CTA then takes many tiles; unset = one or two
- * CTAs per SM).
+ * n == 0 is a no-op.  Testing aids, read at each call: BNBQ_QUANT_MAX_CTAS=<k> caps the kernel's
+ * grid at k CTAs (every CTA then takes many tiles; unset = one or two CTAs per SM);
+ * BNBQ_QUANT_STAGE_FROM=<n> stages aligned fp32 input into shared memory from n elements on
+ * (unset = from 2^26 for 256 codes, 2^28 for 16).
  */
 BNBQ_API bnbq_status bnbq_quantize_blockwise(const float* code, int code_size, const void* A,
                                     bnbq_dtype a_dtype, int64_t n, int blocksize, float* absmax,

@@ -81,6 +81,22 @@ def test_nest_absmax_mean_narrow_scales(nb):
     np.testing.assert_array_equal(parity.to_np(a2).view(np.uint32), a2_or.view(np.uint32))
 
 
+def test_nest_absmax_staged_centred_quantize(monkeypatch):
+    """The centred 8-bit quantize of the scales through the shared-memory stages (forced at this
+    size; by default staging starts at 2^26 scales), with the grid capped so that every CTA takes
+    several tiles."""
+    monkeypatch.setenv("BNBQ_QUANT_STAGE_FROM", "0")
+    monkeypatch.setenv("BNBQ_QUANT_MAX_CTAS", "4")
+    code2 = bq.bnbq_codebook("dynamic_signed")
+    nb = 70001
+    a = _scales(nb, "staged")
+    qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2.to(DEV), a)
+    q_or, a2_or, off_or = oracle.nest_absmax(parity.to_np(a), code2.numpy())
+    assert parity.to_np(off).view(np.uint32)[0] == np.float32(off_or).view(np.uint32)
+    np.testing.assert_array_equal(parity.to_np(a2).view(np.uint32), a2_or.view(np.uint32))
+    np.testing.assert_array_equal(parity.to_np(qabs), q_or)
+
+
 def test_nest_empty_and_equal_scales():
     code2 = bq.bnbq_codebook("dynamic_signed").to(DEV)
     qabs, a2, off = bq.bnbq_quantize_absmax_nested(code2, torch.empty(0, device=DEV))
