@@ -114,6 +114,16 @@ def test_staged_tiles_many_per_cta(code_name, dtype, monkeypatch):
         _check_full(code, x, B)
 
 
+@pytest.mark.parametrize("cap,stage_from", [("abc", "-5"), ("0", "x1"), ("", "")])
+def test_testing_aids_ignore_malformed_values(cap, stage_from, monkeypatch):
+    """Malformed or empty values of the quantize kernel's testing variables leave the defaults in
+    force; results as the oracle's."""
+    monkeypatch.setenv("BNBQ_QUANT_MAX_CTAS", cap)
+    monkeypatch.setenv("BNBQ_QUANT_STAGE_FROM", stage_from)
+    x = sweep_input(50_000 + 11, torch.float32, f"aids-{cap}-{stage_from}")
+    _check_full(_codes()["signed"], x, 2048)
+
+
 @pytest.mark.parametrize("code_name", ["unsigned", "linear"])
 def test_other_codebooks(code_name):
     """Unsigned dynamic code (non-negative data) and the linear code (it has a zero midpoint, so
