@@ -351,7 +351,8 @@ def _code_only(text: str) -> str:
 
 
 QUANT_SOURCES = [os.path.join(ROOT, "block_wise_bit_b200", "csrc", f) for f in
-                 ("bnbq_quant.cu", "bnbq_nested.cu", "bnbq_async.cuh", "bnbq_device.cuh", "bnbq_internal.h")]
+                 ("bnbq_quant.cu", "bnbq_nested.cu", "bnbq_async.cuh", "bnbq_device.cuh", "bnbq_internal.h",
+                  "bnbq_search_fma.cuh")]
 
 
 def quant_source_sha() -> str:

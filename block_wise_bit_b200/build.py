@@ -23,7 +23,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(OUT_DIR, "libbnbq.so")
 SOURCES = ["bnbq_api.cu", "bnbq_quant.cu", "bnbq_step.cu", "bnbq_noalloc.cu", "bnbq_nested.cu"]
-HEADERS = ["bnbq_async.cuh", "bnbq_device.cuh", "bnbq_internal.h"]
+HEADERS = ["bnbq_async.cuh", "bnbq_device.cuh", "bnbq_internal.h", "bnbq_search_fma.cuh"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "bnbq.h")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -22,6 +22,7 @@
 #include "bnbq_async.cuh"
 #include "bnbq_device.cuh"
 #include "bnbq_internal.h"
+#include "bnbq_search_fma.cuh"
 
 namespace bnbq {
 namespace {
@@ -131,38 +132,14 @@ __device__ bool stage_one_code(CodeSmem& cs, const float* code, int K, bool with
     return true;
 }
 
-// The signed search with the sign handled on the FMA pipe (this kernel's integer pipe is the
-// busier one): after the table is built, the negative half's entries are raised by 0xffff, so
-// that entry - low16(x) equals the unbiased entry plus the complement 0xffff - low16(x), and
-// entry + low16(x) * (+1 or -1) gives the code for either sign with one integer multiply-add; the
-// sign half's offset is a multiply-add too.  Same results as kSearchSigned for every input;
-// measured 1-1.5% faster for bf16 input.  (The step kernel keeps the unbiased table: there the
-// same change measured 0.9% slower.)
-constexpr int kSearchSignedFma = 5;
-
-__device__ __forceinline__ void bias_negative_half(CodeSmem& cs)
-{
-    for (int i = threadIdx.x; i < kHalf; i += blockDim.x) cs.table[i] += 0xffffu;  // [0, kHalf): x < 0
-}
-
-__device__ __forceinline__ uint32_t nearest_code_word_fma(const CodeSmem& cs, float x)
-{
-    const uint32_t xb = __float_as_uint(x);
-    const int32_t sx = (int32_t)xb >> 31;                                // -1 if x < 0, else 0
-    const uint32_t t = __float_as_uint(fmaxf(fabsf(x), kTinyEdge));     // magnitude (NaN -> 2^-26)
-    const int32_t off = (int32_t)((t >> 14) & 0x3ffcu) + sx * (4 * kHalf);  // 4 * [-kHalf, kHalf)
-    const uint32_t e = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cs.table + kHalf) + off);
-    return e + (xb & 0xffffu) * (uint32_t)(2 * sx + 1);
-}
-
 // Nearest-code word of a normalised value in the kernel's search mode (code in the top byte).
 template <int MODE>
 __device__ __forceinline__ uint32_t code_word(const CodeSmem& cs, float x)
 {
     if constexpr (MODE == kSearchPrefix11)
         return nearest_code_word11(cs.table, x);
-    else if constexpr (MODE == kSearchSignedFma)
-        return nearest_code_word_fma(cs, x);
+    else if constexpr (MODE == kSearchSignedFma)  // measured 1.5-2% faster than kSearchSigned here
+        return nearest_code_word_fma(cs.table + kHalf, x);
     else
         return nearest_code_word<MODE>(cs, x);
 }
@@ -495,7 +472,7 @@ quantize_kernel(const float* __restrict__ code, const void* __restrict__ A, int6
         quantize_run<B, BF16, WIDE, K, kSearchNonNeg, CENTER, STAGED>(cs, fast, A, n, absmax, out, red, flags, center,
                                                                       smem_raw);
     else {
-        bias_negative_half(cs);  // the table is complete: the barrier of the general test above
+        bias_negative_half(cs.table);  // the table is complete: the barrier of the general test above
         __syncthreads();
         quantize_run<B, BF16, WIDE, K, kSearchSignedFma, CENTER, STAGED>(cs, fast, A, n, absmax, out, red, flags,
                                                                          center, smem_raw);

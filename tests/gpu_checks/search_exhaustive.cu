@@ -4,8 +4,10 @@
 //      q = #{ j : x > mid_j },  mid_j = fl32((code_j + code_{j+1}) / 2)  (sum formed in double),
 // with the midpoints formed on the host.  Each search mode is checked where it applies: the
 // one-load rule when no bucket holds two midpoints, the non-negative rule when every code is
-// >= 0, the midpoint walk always, and for a 16-entry codebook the 11-bit-prefix table
-// (build_table11 / nearest_code_word11) when none of its buckets holds two midpoints.
+// >= 0, the midpoint walk always, for a 16-entry codebook the 11-bit-prefix table
+// (build_table11 / nearest_code_word11) when none of its buckets holds two midpoints, and the
+// one-load rule with the sign on the FMA pipe (bnbq_search_fma.cuh: the table's negative half
+// biased, nearest_code_word_fma) wherever the one-load rule applies.
 //
 // Usage: search_exhaustive <codebook file: K raw float32 values> <K>
 // Prints one line per mode and a final status line; exits 0 only if every checked mode matches.
@@ -15,6 +17,7 @@
 #include <vector>
 
 #include "../../block_wise_bit_b200/csrc/bnbq_device.cuh"
+#include "../../block_wise_bit_b200/csrc/bnbq_search_fma.cuh"
 
 namespace {
 
@@ -39,33 +42,48 @@ __global__ void setup(const float* code, int K, float* mid, uint32_t* table, uin
 
 // One pass over every value: the reference count is formed once per value and compared with each
 // search mode that applies (check[m] != 0), mismatches counted per mode.
-__global__ void sweep(const uint32_t* table, const uint32_t* table11, const float* mid, const float* ref_mid, int K,
-                      int4 check, unsigned long long* bad, unsigned* first)
+constexpr int kModes = 5;
+struct Checks {
+    int on[kModes];
+};
+
+// A copy of the table with the negative half biased, for the FMA-pipe search.
+__global__ void bias_copy(const uint32_t* table, uint32_t* biased)
+{
+    for (int i = threadIdx.x; i < bnbq::kTableSize; i += blockDim.x) biased[i] = table[i];
+    __syncthreads();
+    bnbq::bias_negative_half(biased);
+}
+
+__global__ void sweep(const uint32_t* table, const uint32_t* table11, const uint32_t* biased, const float* mid,
+                      const float* ref_mid, int K, Checks check, unsigned long long* bad, unsigned* first)
 {
     __shared__ float rm[256];
     for (int j = threadIdx.x; j < K - 1; j += blockDim.x) rm[j] = ref_mid[j];
     __syncthreads();
     const uint32_t* center = table + bnbq::kHalf;
+    const uint32_t* center_b = biased + bnbq::kHalf;
     const uint64_t total = 2ull * kHalfValues;
-    unsigned long long n[4] = {0, 0, 0, 0};
+    unsigned long long n[kModes] = {0, 0, 0, 0, 0};
     for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
         const uint32_t bits = i < kHalfValues ? (uint32_t)i : 0x80000000u + (uint32_t)(i - kHalfValues);
         const float x = __uint_as_float(bits);
         uint32_t r = 0;
         for (int j = 0; j < K - 1; j++) r += (x > rm[j]) ? 1u : 0u;
-        uint32_t q[4] = {r, r, r, r};
-        if (check.x) q[0] = bnbq::nearest_code_word<bnbq::kSearchSigned>(center, mid, x) >> 24;
-        if (check.y) q[1] = bnbq::nearest_code_word<bnbq::kSearchNonNeg>(center, mid, x) >> 24;
-        if (check.z) q[2] = bnbq::nearest_code_word<bnbq::kSearchGeneral>(center, mid, x) >> 24;
-        if (check.w) q[3] = bnbq::nearest_code_word11(table11, x) >> 24;
+        uint32_t q[kModes] = {r, r, r, r, r};
+        if (check.on[0]) q[0] = bnbq::nearest_code_word<bnbq::kSearchSigned>(center, mid, x) >> 24;
+        if (check.on[1]) q[1] = bnbq::nearest_code_word<bnbq::kSearchNonNeg>(center, mid, x) >> 24;
+        if (check.on[2]) q[2] = bnbq::nearest_code_word<bnbq::kSearchGeneral>(center, mid, x) >> 24;
+        if (check.on[3]) q[3] = bnbq::nearest_code_word11(table11, x) >> 24;
+        if (check.on[4]) q[4] = bnbq::nearest_code_word_fma(center_b, x) >> 24;
 #pragma unroll
-        for (int m = 0; m < 4; m++)
+        for (int m = 0; m < kModes; m++)
             if (q[m] != r) {
                 n[m]++;
                 atomicCAS(&first[m], 0xffffffffu, bits);
             }
     }
-    for (int m = 0; m < 4; m++)
+    for (int m = 0; m < kModes; m++)
         if (n[m]) atomicAdd(&bad[m], n[m]);
 }
 
@@ -91,7 +109,7 @@ int main(int argc, char** argv)
     }
 
     float *d_code = nullptr, *d_mid = nullptr, *d_ref = nullptr;
-    uint32_t *d_table = nullptr, *d_table11 = nullptr;
+    uint32_t *d_table = nullptr, *d_table11 = nullptr, *d_biased = nullptr;
     int* d_flags = nullptr;
     unsigned long long* d_bad = nullptr;
     unsigned* d_first = nullptr;
@@ -99,8 +117,9 @@ int main(int argc, char** argv)
         cudaMalloc(&d_ref, 256 * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&d_table, bnbq::kTableSize * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&d_table11, bnbq::kTable11 * sizeof(uint32_t)) != cudaSuccess ||
-        cudaMalloc(&d_flags, 3 * sizeof(int)) != cudaSuccess || cudaMalloc(&d_bad, 4 * sizeof(*d_bad)) != cudaSuccess ||
-        cudaMalloc(&d_first, 4 * sizeof(*d_first)) != cudaSuccess)
+        cudaMalloc(&d_biased, bnbq::kTableSize * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&d_flags, 3 * sizeof(int)) != cudaSuccess || cudaMalloc(&d_bad, 5 * sizeof(*d_bad)) != cudaSuccess ||
+        cudaMalloc(&d_first, 5 * sizeof(*d_first)) != cudaSuccess)
         return 3;
     cudaMemcpy(d_code, code.data(), K * sizeof(float), cudaMemcpyHostToDevice);
     cudaMemcpy(d_ref, ref_mid.data(), (K - 1) * sizeof(float), cudaMemcpyHostToDevice);
@@ -116,22 +135,23 @@ int main(int argc, char** argv)
            flags[0], flags[1], nonneg ? 1 : 0, flags[2], mids_equal ? "equal" : "DIFFER");
     bool ok = e == cudaSuccess && flags[1] == 0 && mids_equal;
     if (ok) {
-        // the one-load rule where no bucket holds two midpoints, the non-negative rule for a
-        // codebook without negative codes, the midpoint walk always, and for 16 codes the
-        // 11-bit-prefix table where none of its buckets holds two midpoints
-        const int4 check = make_int4(flags[0] == 0 ? 1 : 0, nonneg ? 1 : 0, 1, (K == 16 && flags[2] == 0) ? 1 : 0);
-        cudaMemset(d_bad, 0, 4 * sizeof(*d_bad));
-        cudaMemset(d_first, 0xff, 4 * sizeof(*d_first));
-        sweep<<<148 * 8, 256>>>(d_table, d_table11, d_mid, d_ref, K, check, d_bad, d_first);
+        // the one-load rule where no bucket holds two midpoints (and its FMA-pipe form), the
+        // non-negative rule for a codebook without negative codes, the midpoint walk always, and
+        // for 16 codes the 11-bit-prefix table where none of its buckets holds two midpoints
+        Checks check = {{flags[0] == 0 ? 1 : 0, nonneg ? 1 : 0, 1, (K == 16 && flags[2] == 0) ? 1 : 0,
+                         flags[0] == 0 ? 1 : 0}};
+        bias_copy<<<1, 1024>>>(d_table, d_biased);
+        cudaMemset(d_bad, 0, 5 * sizeof(*d_bad));
+        cudaMemset(d_first, 0xff, 5 * sizeof(*d_first));
+        sweep<<<148 * 8, 256>>>(d_table, d_table11, d_biased, d_mid, d_ref, K, check, d_bad, d_first);
         e = cudaDeviceSynchronize();
-        unsigned long long bad[4] = {~0ull, ~0ull, ~0ull, ~0ull};
-        unsigned first[4] = {0, 0, 0, 0};
+        unsigned long long bad[kModes] = {~0ull, ~0ull, ~0ull, ~0ull, ~0ull};
+        unsigned first[kModes] = {0, 0, 0, 0, 0};
         cudaMemcpy(bad, d_bad, sizeof(bad), cudaMemcpyDeviceToHost);
         cudaMemcpy(first, d_first, sizeof(first), cudaMemcpyDeviceToHost);
-        const char* names[4] = {"signed", "nonneg", "general", "prefix11"};
-        const int on[4] = {check.x, check.y, check.z, check.w};
-        for (int m = 0; m < 4; m++)
-            if (on[m]) {
+        const char* names[kModes] = {"signed", "nonneg", "general", "prefix11", "signed-fma"};
+        for (int m = 0; m < kModes; m++)
+            if (check.on[m]) {
                 printf("mode %s status %s mismatches %llu first %08x\n", names[m], cudaGetErrorString(e), bad[m],
                        first[m]);
                 ok = ok && e == cudaSuccess && bad[m] == 0;

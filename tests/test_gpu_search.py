@@ -1,8 +1,8 @@
 """Exhaustive check of the nearest-code search used by the quantize and step kernels: for each
 built-in codebook, every binary32 in [-1, 1] goes through the bucket search in each mode that
-applies and is compared with a plain count of the midpoints below it (tests/gpu_checks/
-search_exhaustive.cu, built from the library's own device header); about a second per codebook
-on a B200."""
+applies (including the quantize kernel's FMA-pipe form of the signed search) and is compared with
+a plain count of the midpoints below it (tests/gpu_checks/search_exhaustive.cu, built from the
+library's own device headers); about a second per codebook on a B200."""
 import os
 import subprocess
 
@@ -37,3 +37,5 @@ def test_search_exhaustive(checker, tmp_path, kind):
     assert "midpoints equal" in out.stdout and "mode general status no error mismatches 0" in out.stdout
     if code.size == 16:  # the quantize kernel's search for 16 codes
         assert "mode prefix11 status no error mismatches 0" in out.stdout, out.stdout
+    if "mode signed status" in out.stdout:  # the quantize kernel's form of the signed search
+        assert "mode signed-fma status no error mismatches 0" in out.stdout, out.stdout
