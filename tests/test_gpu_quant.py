@@ -97,19 +97,19 @@ def test_sweep_2p20_elementwise(code_name, B, dtype):
     _check_full(code, x, B)
 
 
+@pytest.mark.parametrize("n", [2 ** 20 + 517, 2 ** 20])
 @pytest.mark.parametrize("code_name", ["signed", "nf4"])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_staged_tiles_many_per_cta(code_name, dtype, monkeypatch):
+def test_staged_tiles_many_per_cta(code_name, dtype, n, monkeypatch):
     """Aligned fp32 input goes through the shared-memory stages (forced at this size).  With
     the grid capped at 3 CTAs every CTA takes 43 tiles (each stage refilled about 20 times, its
     barrier phase flipping each time) and one CTA also quantizes the ragged last tile; bf16 input
     (plain loads) takes 21 passes per CTA.  Compared element by element with the oracle, at
-    blocksizes with 4 to 128 threads per block."""
+    blocksizes with 4 to 128 threads per block; and a size of whole tiles (no ragged tile)."""
     monkeypatch.setenv("BNBQ_QUANT_MAX_CTAS", "3")
     monkeypatch.setenv("BNBQ_QUANT_STAGE_FROM", "0")  # staged at this size too (by default from 2^26)
     code = _codes()[code_name]
-    n = 2 ** 20 + 517
-    x = sweep_input(n, dtype, f"staged-{code_name}-{dtype}")
+    x = sweep_input(n, dtype, f"staged-{code_name}-{dtype}-{n}")
     for B in (64, 128, 2048):
         _check_full(code, x, B)
 
